@@ -1,0 +1,217 @@
+// Hilbert-curve token permutation (paper review page, section 三 "HilbertCurve
+// Permutation"; rebuttal page, reply to Weakness 3): visual tokens of a
+// T x H x W grid are reordered along a Hilbert curve so that spatial
+// neighbours share query/key blocks, and the output is put back afterwards.
+//
+// The table is built on the device by walking the curve: every position h of
+// the 2^(n*b) cube is decoded to grid coordinates with Skilling's transpose
+// algorithm ("Programming the Hilbert curve", AIP Conf. Proc. 707, 2004, the
+// index-to-axes direction), positions outside the grid are dropped, and an
+// exclusive scan over the survivors gives each grid token its rank.  The
+// gather / scatter kernels then move whole 16-byte chunks of token rows.
+#include <cstdint>
+
+#include "sparge_internal.h"
+
+namespace sparge {
+namespace {
+
+constexpr int kHilThreads = 256;
+constexpr int kHilPerThread = 4;
+constexpr int kHilPerCta = kHilThreads * kHilPerThread;
+
+struct HilbertGrid {
+  int32_t n;        // curve dimensions (axes of extent > 1)
+  int32_t bits;     // cube side 2^bits
+  int32_t ext[3];   // extents of the curve axes, in (t, y, x) order
+  int32_t mul[3];   // linear-index multiplier of each curve axis
+  int64_t cube;     // 2^(n*bits)
+};
+
+// Curve position -> grid coordinates (transpose form, Gray decode, undo).
+__device__ __forceinline__ bool hilbert_decode(const HilbertGrid& g, int64_t h, int32_t* lin) {
+  uint32_t X[3] = {0, 0, 0};
+  for (int l = 0; l < g.bits; ++l)
+    for (int i = 0; i < g.n; ++i)
+      X[i] |= uint32_t((h >> (l * g.n + g.n - 1 - i)) & 1) << l;
+  uint32_t t = X[g.n - 1] >> 1;
+  for (int i = g.n - 1; i > 0; --i) X[i] ^= X[i - 1];
+  X[0] ^= t;
+  for (uint32_t Q = 2; Q != (1u << g.bits); Q <<= 1) {
+    const uint32_t P = Q - 1;
+    for (int i = g.n - 1; i >= 0; --i) {
+      if (X[i] & Q) {
+        X[0] ^= P;
+      } else {
+        t = (X[0] ^ X[i]) & P;
+        X[0] ^= t;
+        X[i] ^= t;
+      }
+    }
+  }
+  int32_t L = 0;
+  for (int i = 0; i < g.n; ++i) {
+    if (X[i] >= uint32_t(g.ext[i])) return false;
+    L += int32_t(X[i]) * g.mul[i];
+  }
+  *lin = L;
+  return true;
+}
+
+__global__ void hilbert_count_kernel(HilbertGrid g, int32_t* counts) {
+  const int64_t base = int64_t(blockIdx.x) * kHilPerCta;
+  int c = 0;
+  for (int k = 0; k < kHilPerThread; ++k) {
+    const int64_t h = base + int64_t(threadIdx.x) * kHilPerThread + k;
+    int32_t lin;
+    if (h < g.cube && hilbert_decode(g, h, &lin)) ++c;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
+  __shared__ int sh[kHilThreads / 32];
+  if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = c;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int s = 0;
+    for (int i = 0; i < kHilThreads / 32; ++i) s += sh[i];
+    counts[blockIdx.x] = s;
+  }
+}
+
+__global__ void hilbert_scatter_kernel(HilbertGrid g, const int32_t* counts, int32_t ncount,
+                                       int32_t N, int32_t prefix_len, int32_t L, int32_t* perm) {
+  __shared__ int sh[kHilThreads / 32];
+  __shared__ int s_base;
+  // offset of this CTA = survivors of all earlier CTAs
+  int pre = 0;
+  const int upto = min(int(blockIdx.x), ncount);
+  for (int i = threadIdx.x; i < upto; i += kHilThreads) pre += counts[i];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) pre += __shfl_xor_sync(0xffffffffu, pre, o);
+  if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = pre;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int s = 0;
+    for (int i = 0; i < kHilThreads / 32; ++i) s += sh[i];
+    s_base = s;
+  }
+  __syncthreads();
+  // survivors of this thread, then an exclusive scan across the CTA
+  const int64_t base = int64_t(blockIdx.x) * kHilPerCta + int64_t(threadIdx.x) * kHilPerThread;
+  int32_t lin[kHilPerThread];
+  bool in[kHilPerThread];
+  int c = 0;
+  for (int k = 0; k < kHilPerThread; ++k) {
+    const int64_t h = base + k;
+    in[k] = h < g.cube && hilbert_decode(g, h, &lin[k]);
+    c += in[k];
+  }
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int incl = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  __syncthreads();
+  if (lane == 31) sh[w] = incl;
+  __syncthreads();
+  int warp_off = 0;
+  for (int i = 0; i < w; ++i) warp_off += sh[i];
+  int rank = s_base + warp_off + incl - c;
+  for (int k = 0; k < kHilPerThread; ++k) {
+    if (in[k]) {
+      if (rank < L) perm[prefix_len + rank] = prefix_len + lin[k];
+      ++rank;
+    }
+  }
+  // tokens outside the grid keep their place
+  const int64_t stride = int64_t(gridDim.x) * kHilThreads;
+  for (int64_t p = int64_t(blockIdx.x) * kHilThreads + threadIdx.x; p < N; p += stride)
+    if (p < prefix_len || p >= prefix_len + L) perm[p] = int32_t(p);
+}
+
+// Whole-row gather (y[p] = x[perm[p]]) or scatter (y[perm[p]] = x[p]) inside
+// each (batch, head) slab; blockIdx.y is the slab.  Rows are moved as
+// 16-byte vectors; table entries outside [0, N) are skipped.
+__global__ void permute_kernel(const uint4* __restrict__ x, uint4* __restrict__ y, int32_t N,
+                               int32_t vpr, const int32_t* __restrict__ perm, int inverse) {
+  const int64_t slab = int64_t(blockIdx.y) * N * vpr;
+  const int64_t total = int64_t(N) * vpr;
+  for (int64_t t = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
+       t += int64_t(gridDim.x) * blockDim.x) {
+    const int32_t p = int32_t(t / vpr);
+    const int32_t v = int32_t(t - int64_t(p) * vpr);
+    const int32_t q = __ldg(perm + p);
+    if (uint32_t(q) >= uint32_t(N)) continue;
+    if (!inverse)
+      y[slab + int64_t(p) * vpr + v] = __ldg(x + slab + int64_t(q) * vpr + v);
+    else
+      y[slab + int64_t(q) * vpr + v] = __ldg(x + slab + int64_t(p) * vpr + v);
+  }
+}
+
+bool make_grid(int32_t T, int32_t Hg, int32_t Wg, HilbertGrid* g) {
+  const int32_t ext[3] = {T, Hg, Wg};
+  const int32_t mul[3] = {Hg * Wg, Wg, 1};
+  g->n = 0;
+  int32_t mx = 1;
+  for (int a = 0; a < 3; ++a) {
+    if (ext[a] > 1) {
+      g->ext[g->n] = ext[a];
+      g->mul[g->n] = mul[a];
+      ++g->n;
+      if (ext[a] > mx) mx = ext[a];
+    }
+  }
+  g->bits = 0;
+  while ((1 << g->bits) < mx) ++g->bits;
+  if (g->bits == 0) g->bits = 1;
+  if (g->n * g->bits > 30) return false;
+  g->cube = g->n == 0 ? 0 : (int64_t(1) << (g->n * g->bits));
+  return true;
+}
+
+}  // namespace
+
+size_t hilbert_ws_bytes(int32_t T, int32_t Hg, int32_t Wg) {
+  HilbertGrid g;
+  if (T < 1 || Hg < 1 || Wg < 1 || !make_grid(T, Hg, Wg, &g)) return 0;
+  return align256(size_t(cdiv(g.cube, kHilPerCta) + 1) * sizeof(int32_t));
+}
+
+cudaError_t launch_hilbert_index(int32_t N, int32_t prefix_len, int32_t T, int32_t Hg,
+                                 int32_t Wg, int32_t* perm, void* ws, cudaStream_t s) {
+  HilbertGrid g;
+  if (!make_grid(T, Hg, Wg, &g)) return cudaErrorInvalidValue;
+  const int32_t L = T * Hg * Wg;
+  int32_t* counts = static_cast<int32_t*>(ws);
+  // a grid without an axis of extent > 1 has cube 0: the table is the identity
+  const int64_t ctas = g.cube > 0 ? cdiv(g.cube, kHilPerCta) : 0;
+  if (ctas > 0) {
+    hilbert_count_kernel<<<unsigned(ctas), kHilThreads, 0, s>>>(g, counts);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  const int64_t fill_ctas = cdiv(N, kHilThreads);
+  int64_t grid = ctas > fill_ctas ? ctas : fill_ctas;
+  if (grid < 1) grid = 1;
+  hilbert_scatter_kernel<<<unsigned(grid), kHilThreads, 0, s>>>(
+      g, counts, int32_t(ctas), N, prefix_len, g.cube > 0 ? L : 0, perm);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_rows(const void* x, void* y, int64_t BH, int32_t N, int32_t row_bytes,
+                                const int32_t* perm, bool inverse, cudaStream_t s) {
+  const int32_t vpr = row_bytes / 16;
+  const int64_t total = int64_t(N) * vpr;
+  int64_t gx = cdiv(total, 256 * 4);
+  if (gx < 1) gx = 1;
+  if (gx > 65535) gx = 65535;
+  dim3 grid{unsigned(gx), unsigned(BH), 1u};
+  permute_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(x), static_cast<uint4*>(y), N,
+                                      vpr, perm, inverse ? 1 : 0);
+  return cudaGetLastError();
+}
+
+}  // namespace sparge

@@ -1,0 +1,112 @@
+// Internal declarations shared by the host entry points and the kernels:
+// workspace carving and the launchers of each kernel family.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/sparge.h"
+
+namespace sparge {
+
+inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Offsets (bytes) of every region of the caller's workspace.
+struct WsLayout {
+  size_t status;    // int32 status word (kernels OR/CAS error codes in)
+  size_t q_mean;    // [B, Hq, Tm, d] f32
+  size_t k_mean;    // [B, Hkv, Tn, d] f32
+  size_t s_q;       // [B, Hq, Tm] f32
+  size_t s_k;       // [B, Hkv, Tn] f32
+  size_t v16;       // [B, Hkv, N, d] f16 (bf16 I/O only), else npos
+  size_t q_codes;   // [B, Hq, N, d] int8 (qk_int8), else npos
+  size_t k_codes;   // [B, Hkv, N, d] int8
+  size_t dq;        // [B, Hq, Tm] f32
+  size_t dk;        // [B, Hkv, Tn] f32
+  size_t kbar;      // [B, Hkv, d] f32
+  size_t total;
+  static constexpr size_t npos = ~size_t(0);
+};
+
+inline WsLayout ws_layout(const sparge_params_t& p) {
+  WsLayout w{};
+  const int64_t Tm = cdiv(p.N, p.bq), Tn = cdiv(p.N, p.bk);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off += align256(bytes);
+    return o;
+  };
+  w.status = take(256);
+  w.q_mean = take(size_t(p.B) * p.Hq * Tm * p.d * 4);
+  w.k_mean = take(size_t(p.B) * p.Hkv * Tn * p.d * 4);
+  w.s_q = take(size_t(p.B) * p.Hq * Tm * 4);
+  w.s_k = take(size_t(p.B) * p.Hkv * Tn * 4);
+  w.v16 = p.io_dtype == SPARGE_BF16 ? take(size_t(p.B) * p.Hkv * p.N * p.d * 2) : WsLayout::npos;
+  if (p.qk_int8) {
+    w.q_codes = take(size_t(p.B) * p.Hq * p.N * p.d);
+    w.k_codes = take(size_t(p.B) * p.Hkv * p.N * p.d);
+    w.dq = take(size_t(p.B) * p.Hq * Tm * 4);
+    w.dk = take(size_t(p.B) * p.Hkv * Tn * 4);
+    w.kbar = take(size_t(p.B) * p.Hkv * p.d * 4);
+  } else {
+    w.q_codes = w.k_codes = w.dq = w.dk = w.kbar = WsLayout::npos;
+  }
+  w.total = off;
+  return w;
+}
+
+template <typename T>
+inline T* ws_ptr(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+// ------------------------------------------------------------- predict.cu
+struct PredictPtrs {
+  const void* q;
+  const void* k;
+  float* q_mean;
+  float* k_mean;
+  float* s_q;
+  float* s_k;
+  int8_t* q_codes;  // nullable
+  int8_t* k_codes;  // nullable
+  float* dq;
+  float* dk;
+  float* kbar;
+  uint8_t* mask;
+  int32_t* kv_idx;
+  int32_t* kv_cnt;
+};
+cudaError_t launch_predict(const sparge_params_t& p, const PredictPtrs& ptrs, cudaStream_t s);
+cudaError_t launch_mask_compact(const sparge_params_t& p, const uint8_t* mask, int32_t* kv_idx,
+                                int32_t* kv_cnt, cudaStream_t s);
+
+// ------------------------------------------------------------- permute.cu
+size_t hilbert_ws_bytes(int32_t T, int32_t Hg, int32_t Wg);
+cudaError_t launch_hilbert_index(int32_t N, int32_t prefix_len, int32_t T, int32_t Hg,
+                                 int32_t Wg, int32_t* perm, void* ws, cudaStream_t s);
+cudaError_t launch_permute_rows(const void* x, void* y, int64_t BH, int32_t N, int32_t row_bytes,
+                                const int32_t* perm, bool inverse, cudaStream_t s);
+
+// ------------------------------------------------------------- attn_sm100.cu
+struct AttnPtrs {
+  const void* q;        // io dtype, or int8 codes with qk_int8
+  const void* k;        // io dtype, or int8 codes
+  const void* v;        // io dtype (f16) or the f16 copy in ws
+  const void* v_io;     // caller's V (bf16 when a conversion is needed)
+  void* v16;            // conversion target, or nullptr when V is already f16
+  const float* dq;      // qk_int8 block scales
+  const float* dk;
+  const int32_t* kv_idx;
+  const int32_t* kv_cnt;
+  void* o;
+  int32_t* status;
+  sparge_stats_t* stats;
+};
+// Returns cudaErrorNotSupported when no TMA descriptor could be built.
+cudaError_t launch_attention(const sparge_params_t& p, const AttnPtrs& ptrs, cudaStream_t s);
+
+}  // namespace sparge
