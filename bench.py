@@ -1,0 +1,470 @@
+#!/usr/bin/env python
+"""Throughput of the SpargeAttn sparse-attention forward on B200.
+
+One step = the whole hot path on one batch of synthetic input resident in HBM:
+  [Hilbert table + permute Q, K, V]  (grid workloads only)
+  stage 1  sparge_predict_mask       (pool, INT8 quantisation, select)
+  stage 2  sparge_attn_fwd           (fp16 V copy, tcgen05 attention)
+  [inverse permute O]                (grid workloads only)
+The default workload is the 128K causal GQA INT8 configuration
+(B1, Hq32, Hkv8, N131072, d128, bf16 I/O).  The metric is dense-equivalent
+TOPS = 4 N^2 d Hq (halved when causal) / step time.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+Multi-GPU (torchrun): every rank runs an independent replica of the workload
+(weak scaling, no collective on the data path); the timed region is bracketed
+by barriers and the max over ranks is reported.  --impl reference times the
+CPU oracle on rank 0 on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import signal
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import get_workload, make_qkv  # noqa: E402
+
+METRIC = "sparse-attn dense-equiv TOPS at N=128K causal; sparsity; % tensor-core peak"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_kernel_llm_128k.md")
+ATTN_SRC = os.path.join(ROOT, "free_block_sparse_predict_b200", "csrc", "attn_sm100.cu")
+
+
+def dense_equiv_ops(w) -> float:
+    ops = 4.0 * w.N * w.N * w.d * w.Hq * w.B
+    return ops / 2 if w.causal else ops
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+def profiled_traffic():
+    """dram bytes per attention launch from the committed ncu summary, if it
+    was taken on the current kernel source."""
+    if not os.path.exists(PROFILE_SUMMARY):
+        return None
+    text = open(PROFILE_SUMMARY).read()
+    m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    h = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
+    if not m or not h:
+        return None
+    cur = hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()
+    return float(m.group(1)) if h.group(1) == cur else None
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=self.file, stderr=subprocess.DEVNULL, start_new_session=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        try:
+            os.killpg(self.proc.pid, signal.SIGTERM)
+        except ProcessLookupError:
+            pass
+        self.proc.wait(timeout=10)
+        self.file.flush()
+        rows = []
+        with open(self.file.name) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 8:
+                    rows.append(parts)
+        os.unlink(self.file.name)
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[4:8]) if v == "Active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------
+# native arm
+# ----------------------------------------------------------------------------
+
+def run_native(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import free_block_sparse_predict_b200 as fb
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = _workload(args)
+    t = make_qkv(w, seed=0)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float16
+
+    def host(a):
+        x = torch.from_numpy(a)
+        return x.view(torch.bfloat16) if w.dtype == "bf16" else x
+
+    q_h, k_h, v_h = (host(t[x]).pin_memory() for x in ("q", "k", "v"))
+    q, k, v = (x.to(dev) for x in (q_h, k_h, v_h))
+    p = fb.make_params(w.B, w.Hq, w.Hkv, w.N, w.d, w.tau, w.theta, w.lam, causal=w.causal,
+                       qk_int8=w.qk_int8, io_dtype=tdt)
+    ws = fb.workspace(p, dev)
+    mask, idx, cnt, _, _ = fb.predict_outputs(p, dev)
+    o = torch.empty(q.shape, dtype=tdt, device=dev)
+    stats = torch.zeros(5, dtype=torch.int64, device=dev)
+    perm = hws = None
+    qp = kp = vp = op = None
+    if w.grid:
+        perm = torch.empty(w.N, dtype=torch.int32, device=dev)
+        hws = torch.zeros(fb.sparge_hilbert_workspace_bytes(*w.grid), dtype=torch.uint8,
+                          device=dev)
+        qp, kp, vp, op = (torch.empty_like(x) for x in (q, k, v, o))
+    stream = torch.cuda.current_stream(dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    launches_per_step = 0
+
+    def step(qs, ks, vs, os_, timing=None):
+        nonlocal launches_per_step
+        n = 0
+        if w.grid:
+            fb.sparge_hilbert_index(w.N, w.prefix_len, *w.grid, perm, hws, stream)
+            fb.sparge_hilbert_permute(qs, qp, perm, stream)
+            fb.sparge_hilbert_permute(ks, kp, perm, stream)
+            fb.sparge_hilbert_permute(vs, vp, perm, stream)
+            qs, ks, vs, dst = qp, kp, vp, op
+            n += 2 + 3
+        else:
+            dst = os_
+        if timing:
+            timing[0].record(stream)
+        fb.sparge_predict_mask(p, qs, ks, mask, idx, cnt, None, None, ws, stream)
+        n += 4 if w.qk_int8 else 2
+        if timing:
+            timing[1].record(stream)
+        fb.sparge_attn_fwd(p, qs, ks, vs, idx, cnt, dst, ws, stats, stream)
+        n += 2 if w.dtype == "bf16" else 1
+        if timing:
+            timing[2].record(stream)
+        if w.grid:
+            fb.sparge_inverse_permute(op, os_, perm, stream)
+            n += 1
+        launches_per_step = n
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # ---- device-resident timing
+    for _ in range(args.warmup):
+        step(q, k, v, o)
+    torch.cuda.synchronize()
+    stats.zero_()
+    step(q, k, v, o)                       # one counted step for the work counters
+    torch.cuda.synchronize()
+    st = stats.cpu().numpy().astype(np.int64)
+    if fb.sparge_device_status(ws) != 0:
+        raise RuntimeError("device status reported an error")
+
+    sampler = ClockSampler(_gpu_uuid(torch, dev)) if local_rank == 0 or world > 1 else None
+    barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    e0, e1 = ev(), ev()
+    per = [(ev(), ev(), ev()) for _ in range(args.steps)]
+    e0.record(stream)
+    for s in range(args.steps):
+        step(q, k, v, o, per[s])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop() if sampler else None
+    ms_total = e0.elapsed_time(e1)
+    attn_ms = float(np.mean([a.elapsed_time(b) for (_, a, b) in per]))
+    pred_ms = float(np.mean([a.elapsed_time(b) for (a, b, _) in per]))
+    if world > 1:
+        tt = torch.tensor([ms_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_total = float(tt.item())
+    ms_step = ms_total / args.steps
+    ops_step = dense_equiv_ops(w)
+    value = world * ops_step * args.steps / (ms_total * 1e-3) / 1e12
+
+    # ---- end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        for _ in range(2):
+            q.copy_(q_h, non_blocking=True); k.copy_(k_h, non_blocking=True)
+            v.copy_(v_h, non_blocking=True)
+            step(q, k, v, o)
+            o_h.copy_(o, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier()
+        a, b = ev(), ev()
+        a.record(stream)
+        for _ in range(args.steps):
+            q.copy_(q_h, non_blocking=True); k.copy_(k_h, non_blocking=True)
+            v.copy_(v_h, non_blocking=True)
+            step(q, k, v, o)
+            o_h.copy_(o, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = a.elapsed_time(b)
+        if world > 1:
+            tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            e2e_ms = float(tt.item())
+        nb = lambda x: x.numel() * x.element_size()
+        e2e = {"value": round(world * ops_step * args.steps / (e2e_ms * 1e-3) / 1e12, 3),
+               "unit": "TOPS", "h2d_bytes_per_step": nb(q) + nb(k) + nb(v),
+               "d2h_bytes_per_step": nb(o), "ms_per_step": round(e2e_ms / args.steps, 3)}
+
+    if rank != 0:
+        return None
+
+    # ---- work accounting and roofline of the attention kernel
+    tiles, qk_blocks, pv_blocks, pv_slices, skipped = (int(x) for x in st)
+    vis = _visible_blocks(w)
+    blk_flops = 2.0 * w.bq * w.bk * w.d
+    mma_flops = (qk_blocks + pv_blocks) * blk_flops
+    achieved = mma_flops / (attn_ms * 1e-3) / 1e12
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops_sustained"])
+    peak_burst = float(peaks["bf16_tflops"])
+    traffic = profiled_traffic()
+    sparsity = {
+        "mg": round(1.0 - qk_blocks / vis, 6),
+        "pv_slices_skipped": round(skipped / max(1, pv_slices + skipped), 6),
+        "total": round(1.0 - (qk_blocks + pv_slices / 4.0) / (2.0 * vis), 6),
+    }
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TOPS", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8-qk/f16-pv" if w.qk_int8 else ("bf16" if w.dtype == "bf16" else "f16"),
+        "data": "synthetic (seeded generators; no model weights)",
+        "config": {"workload": f"{w.name}: B{w.B} Hq{w.Hq} Hkv{w.Hkv} N{w.N} d{w.d} "
+                               f"{w.dtype} causal={int(w.causal)} int8_qk={int(w.qk_int8)} "
+                               f"tau={w.tau} theta={w.theta} lambda={w.lam}",
+                   "global_batch": w.B * world, "seq_len": w.N,
+                   "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (no flush)" if _bytes(t) > 126e6
+                   else "inputs smaller than L2"},
+        "latency_ms": {"predict": round(pred_ms, 4), "attention": round(attn_ms, 4),
+                       "step": round(ms_step, 4)},
+        "sparsity": sparsity,
+        "work": {"tiles": tiles, "qk_blocks": qk_blocks, "pv_blocks": pv_blocks,
+                 "pv_slices": pv_slices, "skipped_slices": skipped, "visible_blocks": vis},
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                     "traffic": traffic,
+                     "peak_source": f"{peak_src} bf16 sustained (MEASURED_PEAKS.json)",
+                     "frac_of_burst_peak": round(achieved / peak_burst, 4),
+                     "kernel": "attn_kernel (tcgen05), issued MMA flops per launch / launch time"},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        line["cpu_baseline"] = cpu_baseline(w, t, tiles_per_sample=args.cpu_tiles)
+    return line
+
+
+def _workload(args):
+    w = get_workload(args.workload)
+    return w.replace(N=args.seq_len) if args.seq_len > 0 else w
+
+
+def _bytes(t):
+    return sum(t[x].nbytes for x in ("q", "k", "v"))
+
+
+def _gpu_uuid(torch, dev):
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return str(dev.index)
+
+
+def _visible_blocks(w):
+    Tm, Tn = -(-w.N // w.bq), -(-w.N // w.bk)
+    if not w.causal:
+        return Tm * Tn * w.Hq * w.B
+    tot = 0
+    for i in range(Tm):
+        last = min(w.N, (i + 1) * w.bq) - 1
+        tot += min(Tn, last // w.bk + 1)
+    return tot * w.Hq * w.B
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle on a bounded sample
+# ----------------------------------------------------------------------------
+
+def _oracle_sample(w, t, n_tiles, head=0):
+    """Oracle time for head `head`: the whole-sequence predictor prorated to
+    n_tiles tiles, plus attention on n_tiles evenly spaced query tiles.
+    Returns (dense-equivalent ops of those tiles, seconds)."""
+    from oracle import sparge_oracle as orc
+    from synth import to_f64
+    hk = head // (w.Hq // w.Hkv)
+    Q = to_f64(t["q"][:, head:head + 1], w.dtype)
+    K = to_f64(t["k"][:, hk:hk + 1], w.dtype)
+    V = to_f64(t["v"][:, hk:hk + 1], w.dtype)
+    if w.grid:
+        perm = orc.hilbert_permutation(w.N, w.prefix_len, *w.grid)
+        Q, K, V = (orc.permute_tokens(x, perm) for x in (Q, K, V))
+    Tm = -(-w.N // w.bq)
+    t0 = time.perf_counter()
+    pr = orc.predict_mask(Q, K, w.bq, w.bk, w.tau, w.theta, w.causal, w.scale)
+    t_pred = time.perf_counter() - t0
+    idx, cnt = orc.mask_compact(pr["M"])
+    quant = orc.quantize_qk(Q.astype(np.float32), K.astype(np.float32), w.bq, w.bk) \
+        if w.qk_int8 else None
+    tiles = sorted({int(x) for x in np.linspace(0, Tm - 1, n_tiles)})
+    t1 = time.perf_counter()
+    orc.sparse_attention(Q, K, V, idx, cnt, w.bq, w.bk, w.lam, w.causal, w.scale, quant=quant,
+                         tiles=[(0, 0, i) for i in tiles])
+    t_attn = time.perf_counter() - t1
+    pairs = 0
+    for i in tiles:
+        r0, r1 = i * w.bq, min(w.N, (i + 1) * w.bq)
+        pairs += sum((r + 1) if w.causal else w.N for r in range(r0, r1))
+    ops = 4.0 * w.d * pairs
+    return ops, t_attn + t_pred * len(tiles) / Tm, len(tiles)
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [x.get("num_threads", 1) for x in threadpool_info()]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(w, t, tiles_per_sample=32):
+    ops, sec, n = _oracle_sample(w, t, tiles_per_sample)
+    return {"value": round(ops / sec / 1e12, 9), "unit": "TOPS", "cores": _blas_threads(),
+            "kind": "oracle",
+            "sample": f"head 0: float64 oracle predictor over all {w.N} tokens (time prorated "
+                      f"to the sample) + attention on {n} evenly spaced query tiles; "
+                      f"{sec:.1f} s of CPU"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    w = _workload(args)
+    t = make_qkv(w, seed=0)
+    n = max(1, args.ref_tiles)
+    for _ in range(args.warmup):
+        _oracle_sample(w, t, n)
+    tot_ops = tot_s = 0.0
+    for _ in range(args.steps):
+        ops, sec, n_t = _oracle_sample(w, t, n)
+        tot_ops += ops
+        tot_s += sec
+    value = tot_ops / tot_s / 1e12
+    cores = _blas_threads()
+    sample = (f"head 0: float64 oracle predictor over all {w.N} tokens (time prorated) + "
+              f"attention on {n_t} evenly spaced query tiles per step")
+    return {"metric": METRIC, "value": round(value, 9), "unit": "TOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(1e3 * dense_equiv_ops(w) / (value * 1e12), 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic (seeded generators; no model weights)",
+            "config": {"workload": f"{w.name}: B{w.B} Hq{w.Hq} Hkv{w.Hkv} N{w.N} d{w.d} "
+                                   f"{w.dtype} causal={int(w.causal)} int8_qk={int(w.qk_int8)}",
+                       "global_batch": w.B, "seq_len": w.N, "parallelism": "cpu"},
+            "impl": "reference",
+            "cpu_baseline": {"value": round(value, 9), "unit": "TOPS", "cores": cores,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 9), "unit": "TOPS", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("native", "reference"), default="native")
+    ap.add_argument("--workload", default="llm_128k",
+                    choices=("tiny", "image_dit", "video_dit", "llm_32k", "llm_128k"))
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="override N of the workload (profiling a smaller case)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-tiles", type=int, default=32)
+    ap.add_argument("--ref-tiles", type=int, default=4)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "native":
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+    else:
+        if world > 1:
+            import torch
+            import torch.distributed as dist
+            torch.cuda.set_device(local_rank)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local_rank))
+        try:
+            line = run_native(args, rank, world, local_rank)
+        finally:
+            if world > 1:
+                import torch.distributed as dist
+                dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

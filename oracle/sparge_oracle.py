@@ -467,6 +467,7 @@ def sparse_attention(Q: np.ndarray, K: np.ndarray, V: np.ndarray, kv_idx: np.nda
         zero = l <= 0
         st["zero_l_rows"] += int(zero.sum())
         O[b, h, r0:r1] = np.where(zero[:, None], 0.0, Oi / np.where(zero, 1.0, l)[:, None])
+    st["near_rows"] = near
     return O, st
 
 

@@ -100,11 +100,10 @@ def grid_of(w: Workload):
 
 def bf16_bits_from_f32(x: np.ndarray) -> np.ndarray:
     """Round float32 to bf16 (nearest, ties to even) and return the uint16 bits."""
-    x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    lsb = (u >> 16) & 1
-    u = (u + 0x7FFF + lsb) >> 16
-    return u.astype(np.uint16)
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    lsb = (u >> 16) & np.uint32(1)
+    r = (u + (np.uint32(0x7FFF) + lsb)) >> 16
+    return r.astype(np.uint16)
 
 
 def to_f32(a: np.ndarray, dtype: str) -> np.ndarray:
@@ -189,51 +188,76 @@ def _grf_tokens(rng, H, d, prefix_len, grid, corr, pad, noise=0.1):
     return out
 
 
-def _ar1(rng, H, N, d, phi=0.95, sigma=0.3):
-    from scipy.signal import lfilter
-    out = np.empty((H, N, d), dtype=np.float32)
-    stat_sd = sigma / math.sqrt(1.0 - phi * phi)
-    for h in range(H):
-        e = sigma * rng.standard_normal((N, d))
-        e[0] = stat_sd * rng.standard_normal(d)
-        out[h] = lfilter([1.0], [1.0, -phi], e, axis=0)
-    return out
+def _ar1_head(rng, N, d, phi=0.95, sigma=0.3, chunk=256):
+    """One head of x_t = phi x_{t-1} + N(0, sigma^2) per channel, x_0 drawn
+    from the stationary law.  The recurrence runs in chunks (vectorised over
+    chunks and channels) and the chunk carries are added afterwards."""
+    e = rng.standard_normal((N, d), dtype=np.float32)
+    e *= np.float32(sigma)
+    e[0] *= np.float32(1.0 / math.sqrt(1.0 - phi * phi))
+    nc = -(-N // chunk)
+    E = np.zeros((nc * chunk, d), dtype=np.float32)
+    E[:N] = e
+    Y = E.reshape(nc, chunk, d)
+    ph = np.float32(phi)
+    for t in range(1, chunk):
+        Y[:, t] += ph * Y[:, t - 1]
+    carry = np.empty((nc, d), dtype=np.float32)
+    carry[0] = Y[0, -1]
+    phc = np.float32(phi ** chunk)
+    for c in range(1, nc):
+        carry[c] = Y[c, -1] + phc * carry[c - 1]
+    pw = (phi ** np.arange(1, chunk + 1)).astype(np.float32)
+    Y[1:] += pw[None, :, None] * carry[:-1, None, :]
+    return Y.reshape(nc * chunk, d)[:N]
+
+
+def _head(kind, w, seed_seq):
+    rng = np.random.Generator(np.random.PCG64(seed_seq))
+    if kind == "segments":
+        x = _segments(rng, 1, w.N, w.d)[0]
+    elif kind == "grf":
+        L = int(np.prod(w.grid))
+        if w.prefix_len + L != w.N:
+            raise ValueError("grid workload needs N == prefix_len + T*H*W")
+        corr, pad = ((2.0, 4.0, 4.0), (0, 32, 32)) if w.grid[0] == 1 else \
+            ((2.0, 4.0, 4.0), (11, 18, 19))
+        x = _grf_tokens(rng, 1, w.d, w.prefix_len, w.grid, corr, pad)[0]
+    elif kind == "ar1":
+        x = _ar1_head(rng, w.N, w.d)
+    else:
+        raise ValueError(kind)
+    return _store(x, w.dtype)
 
 
 def make_qkv(w: Workload, seed: int = 0):
     """Q [B,Hq,N,d], K, V [B,Hkv,N,d] in the workload's storage dtype.
 
-    Returns a dict with 'q', 'k', 'v' (np.float16, or uint16 bf16 bits), the
-    workload, and for the AR(1) workloads the needle records
-    (kv_head, k_block, q_block).
+    Every (tensor, batch, head) slab draws from its own PCG64 stream spawned
+    from SeedSequence(seed), so slabs are generated in parallel.  Returns a
+    dict with 'q', 'k', 'v' (np.float16, or uint16 bf16 bits), the workload,
+    and for the AR(1) workloads the needle records (kv_head, k_block, q_block).
     """
-    sq, sk, sv = np.random.SeedSequence(seed).spawn(3)
-    rq, rk, rv = (np.random.Generator(np.random.PCG64(s)) for s in (sq, sk, sv))
+    import concurrent.futures as cf
+    import os
+    root = np.random.SeedSequence(seed)
+    sq, sk, sv, sn = root.spawn(4)
     B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
+    sdt = np.float16 if w.dtype == "f16" else np.uint16
     tensors = {}
-    for name, rng, H in (("q", rq, Hq), ("k", rk, Hkv), ("v", rv, Hkv)):
-        per_b = []
-        for _ in range(B):
-            if w.kind == "segments":
-                x = _segments(rng, H, N, d)
-            elif w.kind == "grf":
-                L = int(np.prod(w.grid))
-                if w.prefix_len + L != N:
-                    raise ValueError("grid workload needs N == prefix_len + T*H*W")
-                if w.grid[0] == 1:
-                    corr, pad = (2.0, 4.0, 4.0), (0, 32, 32)
-                else:
-                    corr, pad = (2.0, 4.0, 4.0), (11, 18, 19)
-                x = _grf_tokens(rng, H, d, w.prefix_len, w.grid, corr, pad)
-            elif w.kind == "ar1":
-                x = _ar1(rng, H, N, d)
-            else:
-                raise ValueError(w.kind)
-            per_b.append(_store(x, w.dtype))
-        tensors[name] = np.stack(per_b)
+    jobs = []
+    with cf.ThreadPoolExecutor(max_workers=min(32, os.cpu_count() or 1)) as ex:
+        for name, ss, H in (("q", sq, Hq), ("k", sk, Hkv), ("v", sv, Hkv)):
+            arr = np.empty((B, H, N, d), dtype=sdt)
+            tensors[name] = arr
+            for idx, child in enumerate(ss.spawn(B * H)):
+                b, h = divmod(idx, H)
+                jobs.append((arr, b, h, ex.submit(_head, w.kind, w, child)))
+        for arr, b, h, fut in jobs:
+            arr[b, h] = fut.result()
     needles = []
     if w.kind == "ar1":
-        rn = np.random.Generator(np.random.PCG64(np.random.SeedSequence(seed).spawn(4)[3]))
+        rn = np.random.Generator(np.random.PCG64(sn))
         g = Hq // Hkv
         Tm = -(-N // w.bq)
         Tn = -(-N // w.bk)

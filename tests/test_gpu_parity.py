@@ -1,0 +1,302 @@
+"""GPU parity of every step of the hot path against the CPU oracle.
+
+All calls go through the C ABI (libsparge.so via the ctypes binding).  Masks
+and index work must match bit-exactly (mask entries the oracle marks as
+ambiguous excepted); float outputs must meet the stated tolerances on the
+float32 output mode, and 16-bit outputs must be within one ulp of the oracle
+rounded to the same dtype."""
+import numpy as np
+import pytest
+import torch
+
+import free_block_sparse_predict_b200 as fb
+from oracle import sparge_oracle as orc
+from synth import bf16_bits_from_f32, to_f32
+
+from gpu_common import (INT8_COS, INT8_REL_L1, MAX_ABS, MEAN_REL_L1, compare_rows, dev,
+                        gpu_attention, gpu_compact, gpu_predict, oracle_inputs, params_for,
+                        sample_tiles, tile_rows, to_dev, torch_dense_attention, workload,
+                        ws_regions)
+
+pytestmark = pytest.mark.gpu
+
+
+# ----------------------------------------------------------------------------
+# permutation
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("N,P,grid", [(4608, 512, (1, 64, 64)), (17776, 226, (13, 30, 45)),
+                                      (50, 3, (2, 3, 7)), (9, 0, (1, 1, 9)), (20, 4, (1, 1, 1))])
+def test_hilbert_table_matches_oracle(N, P, grid):
+    T, H, W = grid
+    perm = torch.full((N,), -7, dtype=torch.int32, device=dev())
+    ws = torch.zeros(fb.sparge_hilbert_workspace_bytes(T, H, W), dtype=torch.uint8,
+                     device=dev())
+    fb.sparge_hilbert_index(N, P, T, H, W, perm, ws)
+    assert np.array_equal(perm.cpu().numpy(), orc.hilbert_permutation(N, P, T, H, W))
+
+
+@pytest.mark.parametrize("dtype,d", [(torch.bfloat16, 128), (torch.float16, 64),
+                                     (torch.float32, 64)])
+def test_permute_gathers_and_inverts_exactly(dtype, d):
+    N = 17776
+    perm_np = orc.hilbert_permutation(N, 226, 13, 30, 45)
+    perm = torch.from_numpy(perm_np.astype(np.int32)).to(dev())
+    x = torch.randn(2, 3, N, d, device=dev()).to(dtype)
+    y, z = torch.empty_like(x), torch.empty_like(x)
+    fb.sparge_hilbert_permute(x, y, perm)
+    fb.sparge_inverse_permute(y, z, perm)
+    assert torch.equal(y, x[:, :, torch.from_numpy(perm_np).to(dev())])
+    assert torch.equal(z, x)
+
+
+# ----------------------------------------------------------------------------
+# stage 1: predictor
+# ----------------------------------------------------------------------------
+
+PREDICT_CASES = [("tiny", {}), ("image_dit", {}), ("video_dit", {}), ("llm_32k", {})]
+
+
+@pytest.mark.parametrize("name,over", PREDICT_CASES, ids=[c[0] for c in PREDICT_CASES])
+def test_predict_mask_matches_oracle(name, over):
+    w, t = workload(name, **over)
+    Q, K, _ = oracle_inputs(w, t)
+    perm = None
+    if w.grid:
+        perm = orc.hilbert_permutation(w.N, w.prefix_len, *w.grid)
+        Q, K = orc.permute_tokens(Q, perm), orc.permute_tokens(K, perm)
+    p = params_for(w)
+    q = to_dev(t["q"], w.dtype)
+    k = to_dev(t["k"], w.dtype)
+    if perm is not None:
+        pt = torch.from_numpy(perm.astype(np.int32)).to(dev())
+        qp, kp = torch.empty_like(q), torch.empty_like(k)
+        fb.sparge_hilbert_permute(q, qp, pt)
+        fb.sparge_hilbert_permute(k, kp, pt)
+        q, k = qp, kp
+    ws, mask, idx, cnt, sq, sk = gpu_predict(p, q, k)
+    pr = orc.predict_mask(Q, K, w.bq, w.bk, w.tau, w.theta, w.causal, w.scale)
+    M = mask.cpu().numpy().astype(bool)
+    bad = (M != pr["M"]) & ~pr["amb"]
+    assert not bad.any(), f"{bad.sum()} mask mismatches, first {np.argwhere(bad)[:3]}"
+    assert np.abs(sq.cpu().numpy() - pr["s_q"]).max() < 1e-5
+    assert np.abs(sk.cpu().numpy() - pr["s_k"]).max() < 1e-5
+    # the skip list is the ascending compaction of the GPU mask
+    io, co = orc.mask_compact(M)
+    c = cnt.cpu().numpy()
+    ii = idx.cpu().numpy()
+    assert np.array_equal(c, co)
+    for pos in np.ndindex(*c.shape):
+        assert np.array_equal(ii[pos][:c[pos]], io[pos][:c[pos]])
+    # causal-future blocks never kept
+    assert not (M & ~pr["visible"]).any()
+
+
+def test_predict_mask_llm_128k_full():
+    w, t = workload("llm_128k")
+    Q, K, _ = oracle_inputs(w, t)
+    p = params_for(w)
+    ws, mask, idx, cnt, sq, sk = gpu_predict(p, to_dev(t["q"], w.dtype), to_dev(t["k"], w.dtype))
+    pr = orc.predict_mask(Q, K, w.bq, w.bk, w.tau, w.theta, w.causal, w.scale)
+    M = mask.cpu().numpy().astype(bool)
+    bad = (M != pr["M"]) & ~pr["amb"]
+    assert not bad.any(), f"{bad.sum()} mismatches"
+    assert np.array_equal(cnt.cpu().numpy(), M.sum(-1))
+
+
+@pytest.mark.parametrize("tau,theta", [(1.0, 0.5), (0.3, -1.5), (0.5, 1.5), (0.7, 0.0)])
+def test_predict_hyperparameter_limits(tau, theta):
+    # tau = 1 keeps every finite block, theta > 1 makes every block a fix
+    # block, theta < -1 is pure TopCdf
+    w, t = workload("llm_32k", N=4096, Hq=4, Hkv=2)
+    Q, K, _ = oracle_inputs(w, t)
+    p = params_for(w, tau=tau, theta=theta)
+    ws, mask, idx, cnt, sq, sk = gpu_predict(p, to_dev(t["q"], w.dtype), to_dev(t["k"], w.dtype))
+    pr = orc.predict_mask(Q, K, w.bq, w.bk, tau, theta, w.causal, w.scale)
+    M = mask.cpu().numpy().astype(bool)
+    assert not ((M != pr["M"]) & ~pr["amb"]).any()
+    if theta > 1:
+        assert np.array_equal(M[0, 0], pr["visible"])
+
+
+# ----------------------------------------------------------------------------
+# stage 2: attention on the oracle's mask
+# ----------------------------------------------------------------------------
+
+def _attention_case(name, over, tiles_per_head=None, heads=None, **pkw):
+    w, t = workload(name, **over)
+    Q, K, V = oracle_inputs(w, t)
+    pr = orc.predict_mask(Q, K, w.bq, w.bk, w.tau, w.theta, w.causal, w.scale)
+    io, co = orc.mask_compact(pr["M"])
+    p = params_for(w, **pkw)
+    idx, cnt = gpu_compact(p, pr["M"])
+    q, k, v = (to_dev(t[x], w.dtype) for x in ("q", "k", "v"))
+    o, st = gpu_attention(p, q, k, v, idx, cnt)
+    tiles = None
+    if tiles_per_head is not None:
+        tiles = sample_tiles(w, tiles_per_head, heads, needles=t["needles"])
+    O, ost = orc.sparse_attention(Q, K, V, io, co, w.bq, w.bk, pkw.get("lam", w.lam), w.causal,
+                                  w.scale, tiles=tiles)
+    rows = tile_rows(w, tiles) if tiles is not None else None
+    return w, o.cpu().numpy(), O, ost, st, rows
+
+
+ATTN_CASES = [("tiny", {}, None, None), ("image_dit", {}, None, None),
+              ("video_dit", {}, 2, [0, 11, 23]), ("llm_32k", {}, 2, [0, 5, 17, 31])]
+
+
+@pytest.mark.parametrize("name,over,tph,heads", ATTN_CASES, ids=[c[0] for c in ATTN_CASES])
+def test_attention_fp32_output_matches_oracle(name, over, tph, heads):
+    w, o, O, ost, st, rows = _attention_case(name, over, tph, heads)
+    # a lambda decision within 1e-3 of the threshold may flip in float32 and
+    # move a whole 32-row slice: those rows are reported, not compared
+    mx, l1 = compare_rows(o, O, rows, exclude=ost["near_rows"])
+    assert mx <= MAX_ABS and l1 <= MEAN_REL_L1, (mx, l1, ost["near_lambda"])
+    if rows is None:
+        # every tile evaluated: the work counters match the oracle's exactly
+        assert st[1] == ost["qk_blocks"]
+        assert abs(int(st[4]) - ost["skipped_slices"]) <= ost["near_lambda"]
+
+
+def test_attention_16bit_output_within_one_ulp():
+    for name in ("tiny", "image_dit"):
+        w, t = workload(name)
+        Q, K, V = oracle_inputs(w, t)
+        pr = orc.predict_mask(Q, K, w.bq, w.bk, w.tau, w.theta, w.causal, w.scale)
+        io, co = orc.mask_compact(pr["M"])
+        from gpu_common import TD
+        p = params_for(w, o_dtype=TD[w.dtype])
+        idx, cnt = gpu_compact(p, pr["M"])
+        q, k, v = (to_dev(t[x], w.dtype) for x in ("q", "k", "v"))
+        o, _ = gpu_attention(p, q, k, v, idx, cnt, out_dtype=TD[w.dtype])
+        O, _ = orc.sparse_attention(Q, K, V, io, co, w.bq, w.bk, w.lam, w.causal, w.scale)
+        if w.dtype == "bf16":
+            gbits = o.view(torch.int16).cpu().numpy().astype(np.int32)
+            obits = bf16_bits_from_f32(O.astype(np.float32)).view(np.int16).astype(np.int32)
+        else:
+            gbits = o.view(torch.int16).cpu().numpy().astype(np.int32)
+            obits = O.astype(np.float16).view(np.int16).astype(np.int32)
+        # same sign: bit patterns are monotone, so the ulp distance is the difference
+        same = np.sign(gbits) == np.sign(obits)
+        dist = np.where(same, np.abs(gbits - obits), 0)
+        assert dist.max() <= 1, dist.max()
+
+
+@pytest.mark.parametrize("name,over", [("tiny", {}), ("image_dit", {"Hq": 4, "Hkv": 4}),
+                                       ("video_dit", {"Hq": 2, "Hkv": 2}),
+                                       ("llm_32k", {"N": 4096, "Hq": 8, "Hkv": 2}),
+                                       ("llm_32k", {"N": 1000, "Hq": 4, "Hkv": 1, "B": 2})])
+def test_dense_limit_equals_torch_softmax_attention(name, over):
+    # theta > 1 makes every block a fix block and lambda = -inf skips nothing:
+    # the result is plain softmax attention
+    w, t = workload(name, **over)
+    p = params_for(w, theta=2.0, lam=float("-inf"))
+    q, k, v = (to_dev(t[x], w.dtype) for x in ("q", "k", "v"))
+    ws, mask, idx, cnt, _, _ = gpu_predict(p, q, k)
+    o, st = gpu_attention(p, q, k, v, idx, cnt, ws)
+    ref = torch_dense_attention(q, k, v, w.scale, w.causal)
+    err = (o - ref).abs()
+    assert err.max().item() <= MAX_ABS
+    assert (err.sum() / ref.abs().sum()).item() <= MEAN_REL_L1
+    assert st[4] == 0
+
+
+# ----------------------------------------------------------------------------
+# INT8 Q K^T with K smoothing
+# ----------------------------------------------------------------------------
+
+def test_int8_codes_and_scales_match_oracle():
+    w, t = workload("llm_128k", N=4096, Hq=8, Hkv=2)
+    Q, K, _ = oracle_inputs(w, t)
+    p = params_for(w)
+    ws, *_ = gpu_predict(p, to_dev(t["q"], w.dtype), to_dev(t["k"], w.dtype))
+    reg = ws_regions(p)
+    raw = ws.cpu().numpy()
+    nq, nk = Q.size, K.size
+    qc = raw[reg["q_codes"]:reg["q_codes"] + nq].view(np.int8).reshape(Q.shape)
+    kc = raw[reg["k_codes"]:reg["k_codes"] + nk].view(np.int8).reshape(K.shape)
+    dq = raw[reg["dq"]:reg["dq"] + 4 * Q.shape[1] * 32].view(np.float32)
+    qt = orc.quantize_qk(Q.astype(np.float32), K.astype(np.float32), 128, 64)
+    assert np.array_equal(qc, qt["q_codes"])                    # same fp32 decisions
+    assert np.array_equal(dq, qt["dq"].ravel())
+    dk = np.abs(kc.astype(np.int32) - qt["k_codes"].astype(np.int32))
+    assert dk.max() <= 1 and dk.mean() < 1e-3                  # kbar summation order only
+
+
+def test_int8_attention_small_matches_exact_scores():
+    w, t = workload("llm_128k", N=4096, Hq=8, Hkv=2)
+    w_, o, O, ost, st, rows = _attention_case("llm_128k", {"N": 4096, "Hq": 8, "Hkv": 2})
+    l1 = np.abs(o - O).sum() / np.abs(O).sum()
+    cos = (o * O).sum() / np.linalg.norm(o) / np.linalg.norm(O)
+    assert l1 <= INT8_REL_L1 and cos >= INT8_COS, (l1, cos)
+
+
+def test_int8_attention_full_128k_sampled_tiles():
+    w, o, O, ost, st, rows = _attention_case("llm_128k", {}, 1, [0, 13, 31])
+    sel = rows
+    a, b = o[sel].astype(np.float64), O[sel]
+    l1 = np.abs(a - b).sum() / np.abs(b).sum()
+    cos = (a * b).sum() / np.linalg.norm(a) / np.linalg.norm(b)
+    assert l1 <= INT8_REL_L1 and cos >= INT8_COS, (l1, cos)
+
+
+# ----------------------------------------------------------------------------
+# edge cases
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("N,causal", [(1, False), (1, True), (65, True), (129, False),
+                                      (200, True), (1000, False)])
+def test_ragged_and_tiny_lengths(N, causal):
+    w, t = workload("llm_32k", N=max(N, 256), Hq=2, Hkv=1)
+    sl = lambda a: np.ascontiguousarray(a[:, :, :N])
+    q, k, v = (to_dev(sl(t[x]), w.dtype) for x in ("q", "k", "v"))
+    w = w.replace(N=N, causal=causal)
+    p = params_for(w, theta=2.0, lam=float("-inf"))
+    ws, mask, idx, cnt, _, _ = gpu_predict(p, q, k)
+    o, _ = gpu_attention(p, q, k, v, idx, cnt, ws)
+    ref = torch_dense_attention(q, k, v, w.scale, causal)
+    assert (o - ref).abs().max().item() <= MAX_ABS
+
+
+def test_empty_rows_and_custom_masks():
+    # tiles with an empty skip list output 0; fully-future blocks kept by a
+    # custom mask contribute nothing; rows that see no key output 0
+    w, t = workload("llm_32k", N=512, Hq=2, Hkv=1)
+    Q, K, V = oracle_inputs(w, t)
+    M = np.zeros((1, 2, 4, 8), dtype=bool)
+    M[0, 0, 1, :] = True          # includes future blocks 4..7 for tile 1
+    M[0, 0, 2, 3] = True
+    M[0, 1, 3, [1, 6]] = True
+    M[0, 1, 0, 1] = True          # rows 0..63 see no key of block 1
+    p = params_for(w, lam=float("-inf"))
+    idx, cnt = gpu_compact(p, M)
+    q, k, v = (to_dev(t[x], w.dtype) for x in ("q", "k", "v"))
+    o, _ = gpu_attention(p, q, k, v, idx, cnt)
+    io, co = orc.mask_compact(M)
+    O, ost = orc.sparse_attention(Q, K, V, io, co, 128, 64, -np.inf, True, w.scale)
+    on = o.cpu().numpy()
+    assert np.all(on[0, 0, :128] == 0) and np.all(on[0, 1, :64] == 0)
+    assert np.abs(on - O).max() <= MAX_ABS
+
+
+def test_lambda_near_zero_skips_all_but_leading_blocks():
+    w, t = workload("llm_32k", N=2048, Hq=2, Hkv=1)
+    Q, K, V = oracle_inputs(w, t)
+    lam = -1e-3
+    _, o, O, ost, st, _ = _attention_case("llm_32k", {"N": 2048, "Hq": 2, "Hkv": 1}, lam=lam)
+    assert st[4] > 0 and abs(int(st[4]) - ost["skipped_slices"]) <= ost["near_lambda"]
+    mx, l1 = compare_rows(o, O)
+    assert l1 <= 10 * MEAN_REL_L1
+
+
+def test_empty_problems_are_no_ops():
+    w, t = workload("tiny")
+    for kw in (dict(N=0), dict(B=0)):
+        ww = w.replace(**kw)
+        p = params_for(ww)
+        ws = torch.zeros(max(256, fb.sparge_workspace_bytes(p)), dtype=torch.uint8, device=dev())
+        dummy = torch.zeros(16, dtype=torch.float16, device=dev())
+        di = torch.zeros(16, dtype=torch.int32, device=dev())
+        fb.sparge_attn_fwd(p, dummy, dummy, dummy, di, di, dummy, ws)
+        fb.sparge_predict_mask(p, dummy, dummy, di, di, di, None, None, ws)
+    torch.cuda.synchronize()
