@@ -129,9 +129,14 @@ def _attention_case(name, over, tiles_per_head=None, heads=None, **pkw):
     pr = orc.predict_mask(Q, K, w.bq, w.bk, w.tau, w.theta, w.causal, w.scale)
     io, co = orc.mask_compact(pr["M"])
     p = params_for(w, **pkw)
-    idx, cnt = gpu_compact(p, pr["M"])
     q, k, v = (to_dev(t[x], w.dtype) for x in ("q", "k", "v"))
-    o, st = gpu_attention(p, q, k, v, idx, cnt)
+    ws = None
+    if w.qk_int8:
+        # the INT8 codes are written by the predictor into the workspace the
+        # attention then reads
+        ws = gpu_predict(p, q, k)[0]
+    idx, cnt = gpu_compact(p, pr["M"])
+    o, st = gpu_attention(p, q, k, v, idx, cnt, ws)
     tiles = None
     if tiles_per_head is not None:
         tiles = sample_tiles(w, tiles_per_head, heads, needles=t["needles"])
