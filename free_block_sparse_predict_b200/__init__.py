@@ -24,7 +24,7 @@ __all__ = [
     "SpargeError", "SpargeParams", "SpargeStats", "make_params", "lib_path",
     "sparge_workspace_bytes", "sparge_hilbert_workspace_bytes", "sparge_hilbert_index",
     "sparge_hilbert_permute", "sparge_inverse_permute", "sparge_predict_mask",
-    "sparge_mask_compact", "sparge_attn_fwd", "sparge_device_status", "sparge_status_string",
+    "sparge_predict_mask_noalloc", "sparge_mask_compact", "sparge_attn_fwd", "sparge_device_status", "sparge_status_string",
     "workspace", "predict_outputs", "sparge_forward",
 ]
 
@@ -99,6 +99,17 @@ def sparge_predict_mask(params, q, k, mask, kv_idx, kv_cnt, s_q, s_k, ws, stream
     _check(lib().sparge_predict_mask(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(mask),
                                      _ptr(kv_idx), _ptr(kv_cnt), _ptr(s_q), _ptr(s_k), _ptr(ws),
                                      ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def sparge_predict_mask_noalloc(params, q, k, mask, kv_idx, kv_cnt, s_q=None, s_k=None,
+                                stream=None) -> None:
+    """sparge_predict_mask without a workspace: for callers that cannot
+    allocate device memory when they call it.  The library's own static
+    device scratch (32 MiB per GPU) holds the intermediates; calls that run
+    concurrently on the GPU share it and race."""
+    _check(lib().sparge_predict_mask_noalloc(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(mask),
+                                             _ptr(kv_idx), _ptr(kv_cnt), _ptr(s_q), _ptr(s_k),
+                                             _stream(stream)))
 
 
 def sparge_mask_compact(params, mask, kv_idx, kv_cnt, stream=None) -> None:

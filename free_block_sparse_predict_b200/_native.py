@@ -44,6 +44,7 @@ SIGNATURES = {
     "sparge_hilbert_permute": (ctypes.c_int, [_V, _V, _I, _I, _I, _I, ctypes.c_int, _V, _V]),
     "sparge_inverse_permute": (ctypes.c_int, [_V, _V, _I, _I, _I, _I, ctypes.c_int, _V, _V]),
     "sparge_predict_mask": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V, _V, _V, _S, _V]),
+    "sparge_predict_mask_noalloc": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V, _V, _V]),
     "sparge_mask_compact": (ctypes.c_int, [_P, _V, _V, _V, _V]),
     "sparge_attn_fwd": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V, _V, _S, _V, _V]),
     "sparge_device_status": (ctypes.c_int, [_V, _V]),

@@ -127,6 +127,30 @@ sparge_status_t sparge_predict_mask(const sparge_params_t* p, const void* q, con
                                     uint8_t* mask, int32_t* kv_idx, int32_t* kv_cnt, float* s_q,
                                     float* s_k, void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* sparge_predict_mask without a workspace, for callers that cannot allocate
+ * device memory at call time and have no workspace to pass in (a plugin whose
+ * host framework owns every device buffer, a serving loop that must not call
+ * the allocator after start-up).  The paper has no counterpart: this is a
+ * deployment variant of the stage-1 predictor above, with the same outputs.
+ * Its scratch (pooled block means and self-similarities) lives in one static
+ * 32 MiB device array compiled into the library; every GPU that loads the
+ * library holds that array until the process exits.  The predictor's regions
+ * must fit: 256 + align256(B*Hq*T_m*d*4) + align256(B*Hkv*T_n*d*4)
+ * + align256(B*Hq*T_m*4) + align256(B*Hkv*T_n*4) <= 32 MiB, else the call
+ * returns SPARGE_EWORKSPACE (align256 rounds up to a multiple of 256).
+ * qk_int8 = 1 returns SPARGE_EUNSUPPORTED (the INT8 codes must outlive the
+ * call); parameter sets that sparge_workspace_bytes rejects return
+ * SPARGE_EINVAL.  The first call on each device looks up the array's device
+ * address there (cudaGetSymbolAddress), so make that first call before any
+ * stream capture.  The call allocates nothing.  All calls share the array and
+ * it keeps the last call's contents; each call rewrites every region it reads,
+ * so nothing has to be cleared, but calls whose kernels overlap on the GPU
+ * (unordered streams) race on it. */
+sparge_status_t sparge_predict_mask_noalloc(const sparge_params_t* p, const void* q,
+                                            const void* k, uint8_t* mask, int32_t* kv_idx,
+                                            int32_t* kv_cnt, float* s_q, float* s_k,
+                                            cudaStream_t stream);
+
 /* Compacts a caller-built mask [B, Hq, T_m, T_n] (uint8, nonzero = keep) into
  * the kv_idx / kv_cnt skip list sparge_attn_fwd consumes.  Causal-future
  * blocks are kept if the mask keeps them (the attention masks them anyway). */
