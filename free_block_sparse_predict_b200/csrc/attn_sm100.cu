@@ -91,6 +91,52 @@ __device__ __forceinline__ void report_timeout(int32_t* status, volatile int* ab
   atomicExch(status, int32_t(SPARGE_ETIMEOUT));
 }
 
+// ---- packed float32 pairs (sm_100a f32x2 arithmetic)
+__device__ __forceinline__ uint64_t pack2(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void unpack2(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+// 2^y for y <= 8 on the FMA pipe, for two values at once.  y = n + f with
+// n = round(y) (adding and subtracting 1.5 * 2^23) and f in [-1/2, 1/2];
+// 2^f by the cubic p(f) that minimises the maximum relative error on that
+// interval (Remez exchange; coefficients from exp2_poly.py, relative error
+// 7.5e-5); 2^n by adding n to the exponent field.  y is clamped at -125 so the
+// exponent never leaves the normal range (2^-125 is 0 for every later use).
+__device__ __forceinline__ void exp2_poly2(float y0, float y1, float& r0, float& r1) {
+  constexpr float kC0 = 9.999280572e-01f, kC1 = 6.932609677e-01f;
+  constexpr float kC2 = 2.426111251e-01f, kC3 = 5.517166853e-02f;
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  y0 = fmaxf(y0, -125.f);
+  y1 = fmaxf(y1, -125.f);
+  const uint64_t y = pack2(y0, y1);
+  const uint64_t t = add2(y, pack2(kMagic, kMagic));
+  const uint64_t nn = add2(t, pack2(-kMagic, -kMagic));
+  const uint64_t f = fma2(nn, pack2(-1.f, -1.f), y);
+  uint64_t p = fma2(pack2(kC3, kC3), f, pack2(kC2, kC2));
+  p = fma2(p, f, pack2(kC1, kC1));
+  p = fma2(p, f, pack2(kC0, kC0));
+  float p0, p1, t0, t1;
+  unpack2(p, p0, p1);
+  unpack2(t, t0, t1);
+  r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 template <int D, int MODE>
 __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const __grid_constant__ AttnParams P) {
   using C = Cfg<D, MODE>;
@@ -263,11 +309,24 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const __grid_constant
     bool issued_any = false;
     uint32_t kept_slices = 0, skipped_slices = 0;
     bool ok = true;
+    // skip-list index (and INT8 block scale) one block ahead of their use
+    int j_next = n > 0 ? __ldg(kv_list) : 0;
     for (int t = 0; t < n; ++t) {
       const int sb = t & 1;
+      const int j = j_next;
+      float sc = P.scale_log2;
+      if (MODE == kI8)
+        sc *= dq_i * (uint32_t(j) < uint32_t(P.Tn) ? __ldg(P.dk + bhk * P.Tn + j) : 0.f);
+      if (t + 1 < n) j_next = __ldg(kv_list + t + 1);
+      // keys c < lim of this block exist for this row (past N, causal future
+      // and rows past N are masked)
+      const int key0 = j * kBK;
+      int lim = P.N - key0;
+      if (P.causal) lim = min(lim, row_g - key0 + 1);
+      if (!row_ok || j < 0) lim = 0;
+
       if (!(ok = mbar_wait(&bars->s_full[sb], (t >> 1) & 1, abort, P.status))) break;
       tc_fence_after();
-      const int j = __ldg(kv_list + t);
       uint32_t raw[64];
       {
         uint32_t (&r0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&raw[0]);
@@ -276,26 +335,38 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const __grid_constant
         tmem_ld32(lane_addr + uint32_t(sb * kBK + 32), r1);
         tmem_wait_ld();
       }
-      float s[64];
-      float sc = P.scale_log2;
-      if (MODE == kI8)
-        sc *= dq_i * (uint32_t(j) < uint32_t(P.Tn) ? __ldg(P.dk + bhk * P.Tn + j) : 0.f);
+      // row max on the raw accumulators (sc > 0 preserves the order), by a tree
+      float m_loc;
+      if (MODE == kI8) {
+        if (lim < 64) {
 #pragma unroll
-      for (int c = 0; c < 64; ++c)
-        s[c] = (MODE == kI8 ? float(int32_t(raw[c])) : __uint_as_float(raw[c])) * sc;
-      // masks: keys past N, causal future, rows past N
-      const int key0 = j * kBK;
-      int lim = P.N - key0;                       // keys c < lim exist
-      if (P.causal) lim = min(lim, row_g - key0 + 1);
-      if (!row_ok || j < 0) lim = 0;
-      if (lim < 64) {
+          for (int c = 0; c < 64; ++c)
+            if (c >= lim) raw[c] = 0x80000000u;
+        }
+        int a[32];
 #pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (c >= lim) s[c] = -INFINITY;
+        for (int c = 0; c < 32; ++c) a[c] = max(int32_t(raw[c]), int32_t(raw[c + 32]));
+#pragma unroll
+        for (int w2 = 16; w2 > 0; w2 >>= 1)
+#pragma unroll
+          for (int c = 0; c < w2; ++c) a[c] = max(a[c], a[c + w2]);
+        m_loc = a[0] == INT32_MIN ? -INFINITY : float(a[0]) * sc;
+      } else {
+        if (lim < 64) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (c >= lim) raw[c] = 0xFF800000u;  // -inf
+        }
+        float a[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          a[c] = fmaxf(__uint_as_float(raw[c]), __uint_as_float(raw[c + 32]));
+#pragma unroll
+        for (int w2 = 16; w2 > 0; w2 >>= 1)
+#pragma unroll
+          for (int c = 0; c < w2; ++c) a[c] = fmaxf(a[c], a[c + w2]);
+        m_loc = a[0] * sc;
       }
-      float m_loc = s[0];
-#pragma unroll
-      for (int c = 1; c < 64; ++c) m_loc = fmaxf(m_loc, s[c]);
       const float m_new = fmaxf(m_true, m_loc);
       const float diff = (m_loc == -INFINITY) ? -INFINITY : (m_loc - m_new);
       const bool skip = __all_sync(0xffffffffu, diff < P.lam2);
@@ -318,18 +389,51 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const __grid_constant
         if (need_o) l *= alpha;
       }
       if (grow) m_sc = m_new;
-      const float base = (m_sc == -INFINITY) ? 0.f : m_sc;
-      uint32_t pk[32];
-      float rs = 0.f;
+      // P~ = 2^(x * sc - m_sc): one packed FMA per pair, then ex2 on the MUFU
+      // for three columns in four and the FMA-pipe polynomial for the fourth
+      const float nb = (m_sc == -INFINITY) ? 0.f : -m_sc;
+      const uint64_t sc2 = pack2(sc, sc), nb2 = pack2(nb, nb);
+      float pv[64];
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float p0 = ex2_approx(s[2 * c] - base);
-        const float p1 = ex2_approx(s[2 * c + 1] - base);
-        rs += p0 + p1;
-        pk[c] = skip ? 0u : pack_half2(p0, p1);
+      for (int c = 0; c < 64; c += 2) {
+        float x0, x1;
+        if (MODE == kI8) {
+          x0 = float(int32_t(raw[c]));
+          x1 = float(int32_t(raw[c + 1]));
+        } else {
+          x0 = __uint_as_float(raw[c]);
+          x1 = __uint_as_float(raw[c + 1]);
+        }
+        float y0, y1;
+        unpack2(fma2(pack2(x0, x1), sc2, nb2), y0, y1);
+        if ((c & 7) == 6) {
+          exp2_poly2(y0, y1, pv[c], pv[c + 1]);
+        } else {
+          pv[c] = ex2_approx(y0);
+          pv[c + 1] = ex2_approx(y1);
+        }
       }
-      l += rs;
+      if (lim < 64) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (c >= lim) pv[c] = 0.f;
+      }
+      // row sum by a packed tree
+      uint64_t acc[16];
+#pragma unroll
+      for (int c = 0; c < 16; ++c)
+        acc[c] = add2(pack2(pv[2 * c], pv[2 * c + 1]), pack2(pv[2 * c + 32], pv[2 * c + 33]));
+#pragma unroll
+      for (int w2 = 8; w2 > 0; w2 >>= 1)
+#pragma unroll
+        for (int c = 0; c < w2; ++c) acc[c] = add2(acc[c], acc[c + w2]);
+      float rs0, rs1;
+      unpack2(acc[0], rs0, rs1);
+      l += rs0 + rs1;
       m_true = m_new;
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) pk[c] = skip ? 0u : pack_half2(pv[2 * c], pv[2 * c + 1]);
       tmem_st32(lane_addr + uint32_t(sb * kBK), pk);
       tmem_wait_st();
       if (!skip) issued_any = true;
