@@ -71,6 +71,24 @@ def profiled_traffic():
     return float(m.group(1)) if h.group(1) == cur else None
 
 
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity on one rank).  The
+    tensor lives on `device` (the GPU for NCCL, None = CPU for gloo)."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate_tops(world: int, ops_per_step: float, steps: int, max_ms: float) -> float:
+    """Whole-job throughput: every rank's dense-equivalent ops over the
+    slowest rank's time for the timed steps."""
+    return world * ops_per_step * steps / (max_ms * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------------------
 # clocks during the timed region
 # ----------------------------------------------------------------------------
@@ -222,13 +240,10 @@ def run_native(args, rank, world, local_rank):
     ms_total = e0.elapsed_time(e1)
     attn_ms = float(np.mean([a.elapsed_time(b) for (_, a, b) in per]))
     pred_ms = float(np.mean([a.elapsed_time(b) for (a, b, _) in per]))
-    if world > 1:
-        tt = torch.tensor([ms_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms_total = float(tt.item())
+    ms_total = max_over_ranks(ms_total, world, dev)
     ms_step = ms_total / args.steps
     ops_step = dense_equiv_ops(w)
-    value = world * ops_step * args.steps / (ms_total * 1e-3) / 1e12
+    value = aggregate_tops(world, ops_step, args.steps, ms_total)
 
     # ---- end to end through the public API with host buffers
     e2e = None
@@ -251,13 +266,9 @@ def run_native(args, rank, world, local_rank):
         b.record(stream)
         torch.cuda.synchronize()
         barrier()
-        e2e_ms = a.elapsed_time(b)
-        if world > 1:
-            tt = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e2e_ms = float(tt.item())
+        e2e_ms = max_over_ranks(a.elapsed_time(b), world, dev)
         nb = lambda x: x.numel() * x.element_size()
-        e2e = {"value": round(world * ops_step * args.steps / (e2e_ms * 1e-3) / 1e12, 3),
+        e2e = {"value": round(aggregate_tops(world, ops_step, args.steps, e2e_ms), 3),
                "unit": "TOPS", "h2d_bytes_per_step": nb(q) + nb(k) + nb(v),
                "d2h_bytes_per_step": nb(o), "ms_per_step": round(e2e_ms / args.steps, 3)}
 

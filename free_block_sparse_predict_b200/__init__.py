@@ -24,7 +24,7 @@ __all__ = [
     "SpargeError", "SpargeParams", "SpargeStats", "make_params", "lib_path",
     "sparge_workspace_bytes", "sparge_hilbert_workspace_bytes", "sparge_hilbert_index",
     "sparge_hilbert_permute", "sparge_inverse_permute", "sparge_predict_mask",
-    "sparge_predict_mask_noalloc", "sparge_mask_compact", "sparge_attn_fwd", "sparge_device_status", "sparge_status_string",
+    "sparge_predict_mask_noalloc", "sparge_mask_compact", "sparge_attn_fwd", "sparge_device_status", "sparge_selftest_wait_timeout", "sparge_status_string",
     "workspace", "predict_outputs", "sparge_forward",
 ]
 
@@ -125,6 +125,12 @@ def sparge_attn_fwd(params, q, k, v, kv_idx, kv_cnt, o, ws, stats=None, stream=N
 
 def sparge_device_status(ws, stream=None) -> int:
     return int(lib().sparge_device_status(_ptr(ws), _stream(stream)))
+
+
+def sparge_selftest_wait_timeout(ws, stream=None) -> None:
+    """Runs the unsatisfiable bounded wait; sparge_device_status then reports
+    SPARGE_ETIMEOUT (4)."""
+    _check(lib().sparge_selftest_wait_timeout(_ptr(ws), _stream(stream)))
 
 
 def sparge_status_string(code: int) -> str:

@@ -48,6 +48,7 @@ SIGNATURES = {
     "sparge_mask_compact": (ctypes.c_int, [_P, _V, _V, _V, _V]),
     "sparge_attn_fwd": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V, _V, _S, _V, _V]),
     "sparge_device_status": (ctypes.c_int, [_V, _V]),
+    "sparge_selftest_wait_timeout": (ctypes.c_int, [_V, _V]),
     "sparge_status_string": (ctypes.c_char_p, [ctypes.c_int]),
 }
 

@@ -7,10 +7,11 @@
 //
 // The array is a fixed kNoAllocScratchBytes (32 MiB) per GPU; every GPU that
 // loads the library holds it until the process exits.  All calls share it and
-// it keeps the last call's contents: every region is completely rewritten by
-// the pooling kernel before any kernel reads it, so nothing needs clearing,
-// but two calls whose kernels overlap on the GPU (different streams, no
-// ordering between them) race on it.
+// it keeps the last call's contents: the status word of the kernels' bounded
+// waits is cleared at the start of every call, every other region is
+// completely rewritten by the pooling kernel before any kernel reads it, and
+// two calls whose kernels overlap on the GPU (different streams, no ordering
+// between them) race on it.
 #include <cstdint>
 #include <mutex>
 
@@ -90,6 +91,9 @@ extern "C" sparge_status_t sparge_predict_mask_noalloc(const sparge_params_t* p,
   x.mask = mask;
   x.kv_idx = kv_idx;
   x.kv_cnt = kv_cnt;
+  // the status word of the kernels' bounded waits must start at zero
+  x.status = ws_ptr<int32_t>(scratch, L.status);
+  if (cudaMemsetAsync(x.status, 0, sizeof(int32_t), stream) != cudaSuccess) return SPARGE_ECUDA;
   if (launch_predict(*p, x, stream) != cudaSuccess) return SPARGE_ECUDA;
   const int64_t Tm = cdiv(p->N, p->bq), Tn = cdiv(p->N, p->bk);
   if (s_q != nullptr && cudaMemcpyAsync(s_q, x.s_q, size_t(p->B) * p->Hq * Tm * 4,

@@ -1,13 +1,13 @@
 // Stage 1 of SpargeAttn: the sparse-block predictor (paper review page,
 // section 三, Eq. 4-9 and Algorithm 1 steps 2-5).
 //
-//   pool_kernel     one pass over Q and K (HBM bound): per block the mean
-//                   token (Eq. 4, 5) and the self-similarity CosSim (Eq. 6,
-//                   read as the mean of the block's token cosine matrix), via
-//                   mean_{a,b} xh_a.xh_b = |sum_a xh_a|^2 / n^2.  With INT8 it
-//                   also quantises Q per block (Algorithm 1 step 2).
+//   pool_warp_kernel<.., 0>  one pass over Q and K (HBM bound), one warp per
+//                   block: the mean token (Eq. 4, 5) and the self-similarity
+//                   CosSim (Eq. 6, read as the mean of the block's token cosine
+//                   matrix), via mean_{a,b} xh_a.xh_b = |sum_a xh_a|^2 / n^2.
+//                   With INT8 it also quantises Q per block (Algorithm 1 step 2).
 //   kbar_kernel     per-head mean of K from the block means (K smoothing).
-//   quant_k_kernel  per-block INT8 of K - kbar (second pass over K).
+//   pool_warp_kernel<.., 1>  per-block INT8 of K - kbar (second pass over K).
 //   select_kernel   per query block: S_hat = scale q_i k^T with -inf columns
 //                   (Eq. 7), row softmax, TopCdf(tau) (Eq. 8) by an exact
 //                   value-threshold bisection, the fix-block rule (Eq. 9), and
@@ -15,9 +15,11 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <algorithm>
 #include <cfloat>
 #include <cstdint>
 
+#include "sm100_ptx.cuh"
 #include "sparge_internal.h"
 
 namespace sparge {
@@ -41,7 +43,41 @@ __device__ __forceinline__ void unpack8(const uint4& raw, float (&x)[8], bool bf
   }
 }
 
-__device__ __forceinline__ uint4 ld_nc_16(const void* p) {
+// code = rint(x * inv), inv = 127 / absmax of the block, clamped to +-127
+__device__ __forceinline__ int8_t quant1(float x, float inv) {
+  float v = rintf(__fmul_rn(x, inv));
+  v = fminf(127.f, fmaxf(-127.f, v));
+  return static_cast<int8_t>(v);
+}
+
+__device__ __forceinline__ uint2 pack_codes(const float (&x)[8], float inv) {
+  uint32_t lo = 0, hi = 0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) lo |= (uint32_t)(uint8_t)quant1(x[e], inv) << (8 * e);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) hi |= (uint32_t)(uint8_t)quant1(x[4 + e], inv) << (8 * e);
+  return make_uint2(lo, hi);
+}
+
+struct PoolArgs {
+  const void* q;
+  const void* k;
+  int32_t N, bq, bk, Tm, Tn;
+  int64_t nQblocks;  // B*Hq*Tm: Q blocks come first in the pooling pass
+  int64_t nblocks;   // blocks this pass visits
+  float* q_mean;
+  float* k_mean;
+  float* s_q;
+  float* s_k;
+  int8_t* q_codes;   // nullable: quantise Q in the pooling pass
+  float* dq;
+  const float* kbar; // INT8 pass over K - kbar
+  int8_t* k_codes;
+  float* dk;
+  int32_t* status;
+};
+
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
   uint4 r;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
@@ -49,212 +85,150 @@ __device__ __forceinline__ uint4 ld_nc_16(const void* p) {
   return r;
 }
 
-__device__ __forceinline__ int8_t quant1(float x, float delta) {
-  if (!(delta > 0.f)) return 0;
-  float v = rintf(__fdiv_rn(x, delta));
-  v = fminf(127.f, fmaxf(-127.f, v));
-  return static_cast<int8_t>(v);
-}
-
-__device__ __forceinline__ uint2 pack_codes(const float (&x)[8], float delta) {
-  uint32_t lo = 0, hi = 0;
-#pragma unroll
-  for (int e = 0; e < 4; ++e) lo |= (uint32_t)(uint8_t)quant1(x[e], delta) << (8 * e);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) hi |= (uint32_t)(uint8_t)quant1(x[4 + e], delta) << (8 * e);
-  return make_uint2(lo, hi);
-}
-
-template <typename F>
-__device__ __forceinline__ float block_reduce(float v, F op, float* sh) {
-  // 256 threads; sh holds >= 8 floats
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
-  const int w = threadIdx.x >> 5;
-  __syncthreads();
-  if ((threadIdx.x & 31) == 0) sh[w] = v;
-  __syncthreads();
-  float r = sh[0];
-#pragma unroll
-  for (int i = 1; i < kPoolThreads / 32; ++i) r = op(r, sh[i]);
-  return r;
-}
-
-struct PoolArgs {
-  const void* q;
-  const void* k;
-  int32_t N, bq, bk, Tm, Tn;
-  int64_t nQblocks;  // B*Hq*Tm
-  float* q_mean;
-  float* k_mean;
-  float* s_q;
-  float* s_k;
-  int8_t* q_codes;  // nullable: quantise Q
-  float* dq;
-};
-
-// One CTA per (head, block) of Q, then of K.  Thread (r0, c) owns the 16-byte
-// chunk c of rows r0, r0 + RPP, ...; the CH lanes of a row reduce its norm.
-template <int D, bool BF16>
-__global__ void __launch_bounds__(kPoolThreads) pool_kernel(PoolArgs a) {
-  constexpr int CH = D * 2 / 16;
-  constexpr int RPP = kPoolThreads / CH;
-  constexpr int MAXP = 128 / RPP;
-  __shared__ __align__(16) float red_x[RPP][D];
-  __shared__ __align__(16) float red_u[RPP][D];
-  __shared__ float sh[8];
-
-  int64_t bid = blockIdx.x;
-  const bool isQ = bid < a.nQblocks;
-  int64_t bh;
-  int blk, BLK;
-  const uint16_t* src;
-  if (isQ) {
-    bh = bid / a.Tm;
-    blk = int(bid % a.Tm);
-    BLK = a.bq;
-    src = static_cast<const uint16_t*>(a.q);
-  } else {
-    bid -= a.nQblocks;
-    bh = bid / a.Tn;
-    blk = int(bid % a.Tn);
-    BLK = a.bk;
-    src = static_cast<const uint16_t*>(a.k);
-  }
-  const int64_t row0 = bh * a.N + int64_t(blk) * BLK;
+// One warp per block, no shared memory and no CTA barrier: lane (ro, c) owns
+// the 16-byte chunk c of rows ro, ro + RPW, ...  Row norms reduce over the CH
+// lanes of a row, column sums over the RPW row groups at the end.
+//   KIND 0  pooling pass over Q blocks then K blocks: mean token, CosSim by
+//           |sum xhat|^2 / n^2, and with q_codes the INT8 codes of Q.
+//   KIND 1  INT8 pass over K blocks: codes of K - kbar and their scales.
+// The codes are a second, L2-resident read of the block once its absmax is
+// known: code = rint(x * (127 / absmax)), clamped to +-127.
+template <int D, bool BF16, int KIND>
+__global__ void __launch_bounds__(256) pool_warp_kernel(PoolArgs a) {
+  constexpr int CH = D * 2 / 16;          // lanes per row
+  constexpr int RPW = 32 / CH;            // rows per warp pass
+  constexpr int UNROLL = 4;
+  const int lane = threadIdx.x & 31;
+  const int64_t id0 = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (id0 >= a.nblocks) return;
+  int64_t id = id0;
+  const bool isQ = KIND == 0 && id < a.nQblocks;
+  if (KIND == 0 && !isQ) id -= a.nQblocks;
+  const int T = isQ ? a.Tm : a.Tn;
+  const int BLK = isQ ? a.bq : a.bk;
+  const int64_t bh = id / T;
+  const int blk = int(id % T);
   const int rows = min(BLK, a.N - blk * BLK);
-  const int tid = threadIdx.x, c = tid % CH, r0 = tid / CH;
+  const uint16_t* src = static_cast<const uint16_t*>(isQ ? a.q : a.k) +
+                        (bh * a.N + int64_t(blk) * BLK) * D;
+  const int c = lane % CH, ro = lane / CH;
 
-  uint4 raw[MAXP];
+  float kb[8];
+  if (KIND == 1) {
 #pragma unroll
-  for (int p = 0; p < MAXP; ++p) {
-    const int r = r0 + p * RPP;
-    raw[p] = make_uint4(0, 0, 0, 0);
-    if (p * RPP < BLK && r < rows) raw[p] = ld_nc_16(src + (row0 + r) * D + c * 8);
+    for (int e = 0; e < 8; ++e) kb[e] = a.kbar[bh * D + c * 8 + e];
   }
   float sx[8], su[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) sx[e] = su[e] = 0.f;
   float amax = 0.f;
+  for (int r0 = ro; r0 < BLK; r0 += RPW * UNROLL) {
+    uint4 raw[UNROLL];
 #pragma unroll
-  for (int p = 0; p < MAXP; ++p) {
-    float x[8];
-    unpack8(raw[p], x, BF16);
-    float ss = 0.f;
+    for (int u = 0; u < UNROLL; ++u) {
+      const int r = r0 + u * RPW;
+      raw[u] = r < rows ? ld_stream(src + int64_t(r) * D + c * 8) : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+    for (int u = 0; u < UNROLL; ++u) {
+      const bool valid = r0 + u * RPW < rows;
+      float x[8];
+      unpack8(raw[u], x, BF16);
+      if (KIND == 0) {
+        float ss = 0.f;
 #pragma unroll
-    for (int o = CH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float inv = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
+        for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      sx[e] += x[e];
-      su[e] = fmaf(x[e], inv, su[e]);
-      amax = fmaxf(amax, fabsf(x[e]));
+        for (int o = CH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float inv = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          sx[e] += x[e];
+          su[e] = fmaf(x[e], inv, su[e]);
+          amax = fmaxf(amax, fabsf(x[e]));
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          if (valid) amax = fmaxf(amax, fabsf(__fsub_rn(x[e], kb[e])));
+      }
     }
   }
-  *reinterpret_cast<float4*>(&red_x[r0][c * 8]) = make_float4(sx[0], sx[1], sx[2], sx[3]);
-  *reinterpret_cast<float4*>(&red_x[r0][c * 8 + 4]) = make_float4(sx[4], sx[5], sx[6], sx[7]);
-  *reinterpret_cast<float4*>(&red_u[r0][c * 8]) = make_float4(su[0], su[1], su[2], su[3]);
-  *reinterpret_cast<float4*>(&red_u[r0][c * 8 + 4]) = make_float4(su[4], su[5], su[6], su[7]);
-  __syncthreads();
-  float uu = 0.f;
-  if (tid < D) {
-    float X = 0.f, U = 0.f;
-#pragma unroll 4
-    for (int r = 0; r < RPP; ++r) {
-      X += red_x[r][tid];
-      U += red_u[r][tid];
-    }
+  if (KIND == 0) {
+    // column sums over the RPW row groups
+#pragma unroll
+    for (int o = CH; o < 32; o <<= 1)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        sx[e] += __shfl_xor_sync(0xffffffffu, sx[e], o);
+        su[e] += __shfl_xor_sync(0xffffffffu, su[e], o);
+      }
+    float uu = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) uu = fmaf(su[e], su[e], uu);
+#pragma unroll
+    for (int o = CH / 2; o > 0; o >>= 1) uu += __shfl_xor_sync(0xffffffffu, uu, o);
     float* mean = isQ ? a.q_mean : a.k_mean;
-    const int64_t T = isQ ? a.Tm : a.Tn;
-    mean[(bh * T + blk) * D + tid] = X / float(rows);
-    uu = U * U;
+    if (lane < CH) {
+      const float n = float(rows);
+      float4* dst = reinterpret_cast<float4*>(mean + (bh * T + blk) * D + c * 8);
+      dst[0] = make_float4(sx[0] / n, sx[1] / n, sx[2] / n, sx[3] / n);
+      dst[1] = make_float4(sx[4] / n, sx[5] / n, sx[6] / n, sx[7] / n);
+    }
+    if (lane == 0) (isQ ? a.s_q : a.s_k)[bh * T + blk] = uu / (float(rows) * float(rows));
   }
-  const float tot = block_reduce(uu, [](float x, float y) { return x + y; }, sh);
-  if (tid == 0) {
-    const float n = float(rows);
-    if (isQ)
-      a.s_q[bh * a.Tm + blk] = tot / (n * n);
-    else
-      a.s_k[bh * a.Tn + blk] = tot / (n * n);
-  }
-  if (isQ && a.q_codes != nullptr) {
-    const float m = block_reduce(amax, [](float x, float y) { return fmaxf(x, y); }, sh);
-    const float delta = m / 127.0f;
-    if (tid == 0) a.dq[bh * a.Tm + blk] = delta;
+  const bool quantise = KIND == 1 || (isQ && a.q_codes != nullptr);
+  if (!quantise) return;
 #pragma unroll
-    for (int p = 0; p < MAXP; ++p) {
-      const int r = r0 + p * RPP;
-      if (p * RPP < BLK && r < rows) {
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float delta = amax / 127.0f;
+  const float inv = amax > 0.f ? 127.0f / amax : 0.f;
+  if (lane == 0) (KIND == 1 ? a.dk : a.dq)[bh * T + blk] = delta;
+  int8_t* codes = (KIND == 1 ? a.k_codes : a.q_codes) + (bh * a.N + int64_t(blk) * BLK) * D;
+  for (int r0 = ro; r0 < rows; r0 += RPW * UNROLL) {
+    uint4 raw[UNROLL];
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const int r = r0 + u * RPW;
+      raw[u] = r < rows ? *reinterpret_cast<const uint4*>(src + int64_t(r) * D + c * 8)
+                        : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < UNROLL; ++u) {
+      const int r = r0 + u * RPW;
+      if (r < rows) {
         float x[8];
-        unpack8(raw[p], x, BF16);
-        *reinterpret_cast<uint2*>(a.q_codes + (row0 + r) * D + c * 8) = pack_codes(x, delta);
+        unpack8(raw[u], x, BF16);
+        if (KIND == 1) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], kb[e]);
+        }
+        *reinterpret_cast<uint2*>(codes + int64_t(r) * D + c * 8) = pack_codes(x, inv);
       }
     }
   }
 }
 
-// kbar[bh, :] = (sum_j n_j * k_mean[bh, j, :]) / N
-__global__ void kbar_kernel(const float* k_mean, float* kbar, int32_t N, int32_t bk, int32_t Tn,
-                            int32_t D) {
+// kbar[bh, :] = (sum_j n_j * k_mean[bh, j, :]) / N, a fixed-order two-level sum
+template <int D>
+__global__ void __launch_bounds__(1024) kbar_kernel(const float* k_mean, float* kbar, int32_t N,
+                                                    int32_t bk, int32_t Tn) {
+  constexpr int G = 1024 / D;
+  __shared__ float part[G][D];
   const int64_t bh = blockIdx.x;
-  for (int col = threadIdx.x; col < D; col += blockDim.x) {
-    float acc = 0.f;
-    for (int j = 0; j < Tn; ++j) {
-      const int n = min(bk, N - j * bk);
-      acc = fmaf(k_mean[(bh * Tn + j) * D + col], float(n), acc);
-    }
-    kbar[bh * D + col] = acc / float(N);
+  const int g = threadIdx.x / D, col = threadIdx.x % D;
+  float acc = 0.f;
+  for (int j = g; j < Tn; j += G) {
+    const int n = min(bk, N - j * bk);
+    acc = fmaf(k_mean[(bh * Tn + j) * D + col], float(n), acc);
   }
-}
-
-struct QuantKArgs {
-  const void* k;
-  const float* kbar;
-  int8_t* k_codes;
-  float* dk;
-  int32_t N, bk, Tn;
-};
-
-template <int D, bool BF16>
-__global__ void __launch_bounds__(kPoolThreads) quant_k_kernel(QuantKArgs a) {
-  constexpr int CH = D * 2 / 16;
-  constexpr int RPP = kPoolThreads / CH;
-  constexpr int MAXP = 64 / RPP > 0 ? 64 / RPP : 1;
-  __shared__ float sh[8];
-  const int64_t bh = blockIdx.x / a.Tn;
-  const int blk = int(blockIdx.x % a.Tn);
-  const int64_t row0 = bh * a.N + int64_t(blk) * a.bk;
-  const int rows = min(a.bk, a.N - blk * a.bk);
-  const int tid = threadIdx.x, c = tid % CH, r0 = tid / CH;
-  const uint16_t* src = static_cast<const uint16_t*>(a.k);
-  float kb[8];
+  part[g][col] = acc;
+  __syncthreads();
+  if (g == 0) {
+    float s = 0.f;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) kb[e] = a.kbar[bh * D + c * 8 + e];
-  float xs[MAXP][8];
-  float amax = 0.f;
-#pragma unroll
-  for (int p = 0; p < MAXP; ++p) {
-    const int r = r0 + p * RPP;
-    uint4 raw = make_uint4(0, 0, 0, 0);
-    const bool ok = p * RPP < a.bk && r < rows;
-    if (ok) raw = ld_nc_16(src + (row0 + r) * D + c * 8);
-    unpack8(raw, xs[p], BF16);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      xs[p][e] = ok ? __fsub_rn(xs[p][e], kb[e]) : 0.f;
-      amax = fmaxf(amax, fabsf(xs[p][e]));
-    }
-  }
-  const float m = block_reduce(amax, [](float x, float y) { return fmaxf(x, y); }, sh);
-  const float delta = m / 127.0f;
-  if (tid == 0) a.dk[bh * a.Tn + blk] = delta;
-#pragma unroll
-  for (int p = 0; p < MAXP; ++p) {
-    const int r = r0 + p * RPP;
-    if (p * RPP < a.bk && r < rows)
-      *reinterpret_cast<uint2*>(a.k_codes + (row0 + r) * D + c * 8) = pack_codes(xs[p], delta);
+    for (int i = 0; i < G; ++i) s += part[i][col];
+    kbar[bh * D + col] = s / float(N);
   }
 }
 
@@ -435,22 +409,31 @@ cudaError_t predict_impl(const sparge_params_t& p, const PredictPtrs& x, cudaStr
   pa.Tm = int32_t(Tm);
   pa.Tn = int32_t(Tn);
   pa.nQblocks = int64_t(p.B) * p.Hq * Tm;
+  pa.nblocks = pa.nQblocks + int64_t(p.B) * p.Hkv * Tn;
   pa.q_mean = x.q_mean;
   pa.k_mean = x.k_mean;
   pa.s_q = x.s_q;
   pa.s_k = x.s_k;
   pa.q_codes = x.q_codes;
   pa.dq = x.dq;
-  const int64_t nblocks = pa.nQblocks + int64_t(p.B) * p.Hkv * Tn;
-  pool_kernel<D, BF16><<<dim3(unsigned(nblocks)), kPoolThreads, 0, s>>>(pa);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
+  pa.status = x.status;
+  cudaError_t e;
+  const int64_t warps_per_cta = kPoolThreads / 32;
+  pool_warp_kernel<D, BF16, 0>
+      <<<unsigned(cdiv(pa.nblocks, warps_per_cta)), kPoolThreads, 0, s>>>(pa);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (x.k_codes != nullptr) {
-    kbar_kernel<<<unsigned(int64_t(p.B) * p.Hkv), 128, 0, s>>>(x.k_mean, x.kbar, p.N, p.bk,
-                                                               int32_t(Tn), D);
+    kbar_kernel<D><<<unsigned(int64_t(p.B) * p.Hkv), 1024, 0, s>>>(x.k_mean, x.kbar, p.N, p.bk,
+                                                                   int32_t(Tn));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    QuantKArgs qa{x.k, x.kbar, x.k_codes, x.dk, p.N, p.bk, int32_t(Tn)};
-    quant_k_kernel<D, BF16><<<unsigned(int64_t(p.B) * p.Hkv * Tn), kPoolThreads, 0, s>>>(qa);
+    PoolArgs qa = pa;
+    qa.nblocks = int64_t(p.B) * p.Hkv * Tn;
+    qa.nQblocks = 0;
+    qa.kbar = x.kbar;
+    qa.k_codes = x.k_codes;
+    qa.dk = x.dk;
+    pool_warp_kernel<D, BF16, 1>
+        <<<unsigned(cdiv(qa.nblocks, warps_per_cta)), kPoolThreads, 0, s>>>(qa);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   SelectArgs sa{};
@@ -476,8 +459,8 @@ cudaError_t predict_impl(const sparge_params_t& p, const PredictPtrs& x, cudaStr
   e = cudaFuncSetAttribute(select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            int(smem));
   if (e != cudaSuccess) return e;
-  dim3 grid{unsigned(cdiv(Tm, kSelRows)), unsigned(p.Hq), unsigned(p.B)};
-  select_kernel<D><<<grid, 256, smem, s>>>(sa);
+  dim3 sgrid{unsigned(cdiv(Tm, kSelRows)), unsigned(p.Hq), unsigned(p.B)};
+  select_kernel<D><<<sgrid, 256, smem, s>>>(sa);
   return cudaGetLastError();
 }
 

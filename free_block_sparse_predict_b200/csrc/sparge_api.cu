@@ -154,6 +154,7 @@ sparge_status_t sparge_predict_mask(const sparge_params_t* p, const void* q, con
   x.mask = mask;
   x.kv_idx = kv_idx;
   x.kv_cnt = kv_cnt;
+  x.status = ws_ptr<int32_t>(ws, L.status);
   cudaError_t e = launch_predict(*p, x, stream);
   if (e != cudaSuccess) return from_cuda(e);
   const int64_t Tm = cdiv(p->N, p->bq), Tn = cdiv(p->N, p->bk);

@@ -79,6 +79,7 @@ struct PredictPtrs {
   uint8_t* mask;
   int32_t* kv_idx;
   int32_t* kv_cnt;
+  int32_t* status;  // device status word (timeouts of the bounded waits)
 };
 cudaError_t launch_predict(const sparge_params_t& p, const PredictPtrs& ptrs, cudaStream_t s);
 cudaError_t launch_mask_compact(const sparge_params_t& p, const uint8_t* mask, int32_t* kv_idx,

@@ -175,6 +175,14 @@ sparge_status_t sparge_attn_fwd(const sparge_params_t* p, const void* q, const v
  * ws: the workspace of sparge_predict_mask / sparge_attn_fwd. */
 sparge_status_t sparge_device_status(void* ws, cudaStream_t stream);
 
+/* Failure-detection self-test (no counterpart in the paper): launches one
+ * CTA whose time-bounded mbarrier wait -- the same wait the attention kernel
+ * uses -- is on a phase that nothing ever completes.  The wait gives up after
+ * its 1 s limit and writes SPARGE_ETIMEOUT into the status word of ws, which
+ * sparge_device_status then returns (and clears).  Nothing faults, traps or
+ * hangs; the context stays usable.  ws: any workspace of at least 256 bytes. */
+sparge_status_t sparge_selftest_wait_timeout(void* ws, cudaStream_t stream);
+
 /* Static description of a status code (never NULL). */
 const char* sparge_status_string(sparge_status_t s);
 

@@ -40,8 +40,9 @@ design notes):
   R7  A row with l = 0 outputs 0.
   R8  GQA: query head h reads KV head h // (Hq/Hkv).
   R9  INT8: kbar = per-(batch, KV head) float32 mean of K over all tokens;
-      K' = K - kbar in float32; delta = absmax/127 in float32; code =
-      round-half-even(x / delta) with an IEEE float32 divide, clamped to +-127.
+      K' = K - kbar in float32; per block delta = absmax/127 (the dequantisation
+      scale) and inv = 127/absmax, both float32 divides; code =
+      round-half-even(x * inv) with a float32 multiply, clamped to +-127.
       The subtracted kbar shifts each score row by a constant, so no bias term
       ("delta Bias" of Algorithm 1 step 10) is added.  The predictor itself
       pools the original K.
@@ -358,10 +359,10 @@ def quantize_blocks(X32: np.ndarray, b: int):
         r0, r1 = block_rows(N, b, i)
         blk = X32[r0:r1]
         amax = np.float32(np.abs(blk).max()) if blk.size else np.float32(0)
-        dl = np.float32(amax / np.float32(127.0))
-        delta[i] = dl
-        if dl > 0:
-            v = np.rint(blk / dl)          # float32 divide, round half to even
+        delta[i] = np.float32(amax / np.float32(127.0))
+        if amax > 0:
+            inv = np.float32(np.float32(127.0) / amax)
+            v = np.rint(blk * inv)         # float32 multiply, round half to even
             codes[r0:r1] = np.clip(v, -127, 127).astype(np.int8)
     return codes, delta
 
