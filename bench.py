@@ -438,6 +438,141 @@ def run_reference(args, rank, world):
                     "d2h_bytes_per_step": 0}}
 
 
+# ----------------------------------------------------------------------------
+# sweeps: the pages' ablations on the synthetic workloads (one JSON line each)
+# ----------------------------------------------------------------------------
+
+def _measure(w, steps=3, warmup=2, perm=None, want_output=False, seed=0, tensors=None):
+    """Times predict + attention for workload w (grid permutation applied
+    outside the timed region when perm is given).  Returns counters, times and
+    optionally the float32 output and the self-similarities."""
+    import torch
+    import free_block_sparse_predict_b200 as fb
+    dev = torch.device("cuda", 0)
+    t = tensors if tensors is not None else make_qkv(w, seed=seed)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float16
+
+    def dv(a):
+        x = torch.from_numpy(a).to(dev)
+        return x.view(torch.bfloat16) if w.dtype == "bf16" else x
+    q, k, v = dv(t["q"]), dv(t["k"]), dv(t["v"])
+    if perm is not None:
+        pt = torch.from_numpy(perm.astype(np.int32)).to(dev)
+        q2, k2, v2 = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        fb.sparge_hilbert_permute(q, q2, pt)
+        fb.sparge_hilbert_permute(k, k2, pt)
+        fb.sparge_hilbert_permute(v, v2, pt)
+        q, k, v = q2, k2, v2
+    p = fb.make_params(w.B, w.Hq, w.Hkv, w.N, w.d, w.tau, w.theta, w.lam, causal=w.causal,
+                       qk_int8=w.qk_int8, io_dtype=tdt,
+                       o_dtype=torch.float32 if want_output else tdt)
+    ws = fb.workspace(p, dev)
+    mask, idx, cnt, sq, sk = fb.predict_outputs(p, dev)
+    o = torch.empty(q.shape, dtype=torch.float32 if want_output else tdt, device=dev)
+    stats = torch.zeros(5, dtype=torch.int64, device=dev)
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    for _ in range(warmup):
+        fb.sparge_predict_mask(p, q, k, mask, idx, cnt, sq, sk, ws)
+        fb.sparge_attn_fwd(p, q, k, v, idx, cnt, o, ws)
+    torch.cuda.synchronize()
+    a, b, c = ev(), ev(), ev()
+    pm = am = 0.0
+    for i in range(steps):
+        a.record()
+        fb.sparge_predict_mask(p, q, k, mask, idx, cnt, sq, sk, ws)
+        b.record()
+        fb.sparge_attn_fwd(p, q, k, v, idx, cnt, o, ws, stats if i == 0 else None)
+        c.record()
+        torch.cuda.synchronize()
+        pm += a.elapsed_time(b)
+        am += b.elapsed_time(c)
+    st = [int(x) for x in stats.cpu()]
+    vis = _visible_blocks(w)
+    step_ms = (pm + am) / steps
+    out = {"N": w.N, "tau": w.tau, "theta": w.theta, "lambda": w.lam,
+           "predict_ms": round(pm / steps, 4), "attention_ms": round(am / steps, 4),
+           "tops": round(dense_equiv_ops(w) / (step_ms * 1e-3) / 1e12, 2),
+           "sparsity": {"mg": round(1 - st[1] / vis, 5),
+                        "pv_slices_skipped": round(st[4] / max(1, st[3] + st[4]), 5),
+                        "total": round(1 - (st[1] + st[3] / 4) / (2 * vis), 5)}}
+    extra = {"o": o.float() if want_output else None, "s_q": sq, "s_k": sk, "perm_q": q}
+    return out, extra
+
+
+def run_sweep(args):
+    import torch
+    kind = args.sweep
+    base = _workload(args)
+    lines = []
+    if kind == "table6":
+        # Table 6 of the paper review: only M_g (lambda = -inf), only M_pv
+        # (theta > 1: every block computed), and both; at the configuration's
+        # theta and at lower theta values that make blocks selective
+        for theta in (base.theta, 0.3, 0.0):
+            for name, over in (("only_mg", {"lam": float("-inf")}), ("only_mpv", {"theta": 2.0}),
+                               ("both", {})):
+                w = base.replace(**{"theta": theta, **over})
+                r, _ = _measure(w)
+                r.update(sweep="table6", strategy=name, theta_setting=theta)
+                lines.append(r)
+    elif kind == "length":
+        for n in (8192, 16384, 32768, 65536, 131072):
+            w = base.replace(N=n)
+            r, _ = _measure(w)
+            r.update(sweep="length")
+            lines.append(r)
+    elif kind == "tau":
+        # speed against sparsity (Fig. 9 of the paper review) with every block
+        # selective (theta = -1) so that TopCdf alone sets the block mask
+        for tau in (0.3, 0.5, 0.7, 0.8, 0.9, 0.95, 0.99, 1.0):
+            w = base.replace(tau=tau, theta=-1.0)
+            r, _ = _measure(w)
+            r.update(sweep="tau")
+            lines.append(r)
+    elif kind == "permutation":
+        # Table 4 of the paper review on the synthetic video grid: block
+        # self-similarity, L1 error against dense attention, and sparsity
+        import free_block_sparse_predict_b200 as fb
+        w = get_workload(args.workload if args.workload in ("image_dit", "video_dit")
+                         else "video_dit")
+        t = make_qkv(w, seed=0)
+        T, H, W = w.grid
+        P, L = w.prefix_len, T * H * W
+        rng = np.random.default_rng(0)
+        lin = np.arange(L)
+        tt, rem = np.divmod(lin, H * W)
+        yy, xx = np.divmod(rem, W)
+        perms = {
+            "random": np.concatenate([np.arange(P), P + rng.permutation(L)]),
+            "rowmajor": np.arange(w.N),
+            "timemajor": np.concatenate([np.arange(P), P + np.lexsort((tt, xx, yy))]),
+        }
+        dev = torch.device("cuda", 0)
+        hp = torch.empty(w.N, dtype=torch.int32, device=dev)
+        hws = torch.zeros(fb.sparge_hilbert_workspace_bytes(T, H, W), dtype=torch.uint8,
+                          device=dev)
+        fb.sparge_hilbert_index(w.N, P, T, H, W, hp, hws)
+        perms["hilbert"] = hp.cpu().numpy()
+        dense_w = w.replace(theta=2.0, lam=float("-inf"))
+        for name, perm in perms.items():
+            _, dense = _measure(dense_w, steps=1, warmup=1, perm=perm, want_output=True, tensors=t)
+            # the configuration's theta, and a lower one at which blocks can be selective
+            for theta in (w.theta, 0.3):
+                r, sp = _measure(w.replace(theta=theta), steps=3, warmup=1, perm=perm,
+                                 want_output=True, tensors=t)
+                O, O2 = dense["o"], sp["o"]
+                l1 = float((O - O2).abs().sum() / O.abs().sum())
+                nq = P // w.bq
+                nk = P // w.bk
+                r.update(sweep="permutation", permutation=name,
+                         sim_q=round(float(sp["s_q"][..., nq:].mean()), 4),
+                         sim_k=round(float(sp["s_k"][..., nk:].mean()), 4), l1=round(l1, 5))
+                lines.append(r)
+    for r in lines:
+        r["workload"] = base.name if kind != "permutation" else r.get("workload", "video_dit")
+        print(json.dumps(r), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -452,12 +587,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-tiles", type=int, default=32)
     ap.add_argument("--ref-tiles", type=int, default=4)
+    ap.add_argument("--sweep", choices=("table6", "length", "tau", "permutation"), default=None,
+                    help="run an ablation sweep instead of the benchmark (one JSON line per point)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":
         args.warmup = 3
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.impl == "reference":
         line = run_reference(args, rank, world)
     else:
