@@ -3,7 +3,8 @@
 
 One step = the whole hot path on one batch of synthetic input resident in HBM:
   [Hilbert table + permute Q, K, V]  (grid workloads only)
-  stage 1  sparge_predict_mask       (pool, INT8 quantisation, select)
+  stage 1  sparge_predict_pool        (block means, CosSim, INT8 codes: HBM bound)
+           sparge_predict_select      (S_hat, TopCdf, fix rule, skip list)
   stage 2  sparge_attn_fwd           (fp16 V copy, tcgen05 attention)
   [inverse permute O]                (grid workloads only)
 The default workload is the 128K causal GQA INT8 configuration
@@ -47,6 +48,27 @@ ATTN_SRC = os.path.join(ROOT, "free_block_sparse_predict_b200", "csrc", "attn_sm
 def dense_equiv_ops(w) -> float:
     ops = 4.0 * w.N * w.N * w.d * w.Hq * w.B
     return ops / 2 if w.causal else ops
+
+
+def pool_bytes(w) -> float:
+    """Algorithmic HBM bytes of one predictor pooling stage: one read of Q and
+    K, the block means and self-similarities written, and with INT8 the Q codes,
+    k-bar (from the K means), a second read of K and the K codes."""
+    es = 2
+    Tm, Tn = -(-w.N // w.bq), -(-w.N // w.bk)
+    bq_, bk_ = w.B * w.Hq, w.B * w.Hkv
+    b = (bq_ + bk_) * w.N * w.d * es + (bq_ * Tm + bk_ * Tn) * (w.d + 1) * 4
+    if w.qk_int8:
+        b += bq_ * w.N * w.d + bq_ * Tm * 4                       # Q codes, scales
+        b += bk_ * Tn * w.d * 4                                   # k-bar from the K means
+        b += bk_ * w.N * w.d * es + bk_ * w.N * w.d + bk_ * Tn * 4  # K again, codes, scales
+    return float(b)
+
+
+def fp32_peak_tflops(peaks) -> float:
+    """FP32 FMA peak derived from the unit counts: 148 SMs x 128 FP32 lanes x
+    2 flops x the measured maximum SM clock."""
+    return 148 * 128 * 2 * float(peaks.get("sm_max_mhz", 1965.0)) * 1e6 / 1e12
 
 
 def load_peaks():
@@ -194,14 +216,18 @@ def run_native(args, rank, world, local_rank):
             dst = os_
         if timing:
             timing[0].record(stream)
-        fb.sparge_predict_mask(p, qs, ks, mask, idx, cnt, None, None, ws, stream)
-        n += 4 if w.qk_int8 else 2
+        fb.sparge_predict_pool(p, qs, ks, ws, stream)
+        n += 4 if w.qk_int8 else 1
         if timing:
             timing[1].record(stream)
+        fb.sparge_predict_select(p, mask, idx, cnt, None, None, ws, stream)
+        n += 1
+        if timing:
+            timing[2].record(stream)
         fb.sparge_attn_fwd(p, qs, ks, vs, idx, cnt, dst, ws, stats, stream)
         n += 2 if w.dtype == "bf16" else 1
         if timing:
-            timing[2].record(stream)
+            timing[3].record(stream)
         if w.grid:
             fb.sparge_inverse_permute(op, os_, perm, stream)
             n += 1
@@ -229,7 +255,7 @@ def run_native(args, rank, world, local_rank):
         sampler.start()
         time.sleep(0.3)
     e0, e1 = ev(), ev()
-    per = [(ev(), ev(), ev()) for _ in range(args.steps)]
+    per = [(ev(), ev(), ev(), ev()) for _ in range(args.steps)]
     e0.record(stream)
     for s in range(args.steps):
         step(q, k, v, o, per[s])
@@ -238,8 +264,10 @@ def run_native(args, rank, world, local_rank):
     barrier()
     clocks = sampler.stop() if sampler else None
     ms_total = e0.elapsed_time(e1)
-    attn_ms = float(np.mean([a.elapsed_time(b) for (_, a, b) in per]))
-    pred_ms = float(np.mean([a.elapsed_time(b) for (a, b, _) in per]))
+    pool_ms = float(np.mean([a.elapsed_time(b) for (a, b, _, _) in per]))
+    sel_ms = float(np.mean([a.elapsed_time(b) for (_, a, b, _) in per]))
+    attn_ms = float(np.mean([a.elapsed_time(b) for (_, _, a, b) in per]))
+    pred_ms = pool_ms + sel_ms
     ms_total = max_over_ranks(ms_total, world, dev)
     ms_step = ms_total / args.steps
     ops_step = dense_equiv_ops(w)
@@ -285,6 +313,10 @@ def run_native(args, rank, world, local_rank):
     peak = float(peaks["bf16_tflops_sustained"])
     peak_burst = float(peaks["bf16_tflops"])
     traffic = profiled_traffic()
+    pbytes = pool_bytes(w)
+    hbm_peak = float(peaks["hbm_gbs"])
+    sel_flops = 2.0 * w.d * _visible_pairs(w)
+    fp32_peak = fp32_peak_tflops(peaks)
     sparsity = {
         "mg": round(1.0 - qk_blocks / vis, 6),
         "pv_slices_skipped": round(skipped / max(1, pv_slices + skipped), 6),
@@ -303,8 +335,23 @@ def run_native(args, rank, world, local_rank):
                    "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (no flush)" if _bytes(t) > 126e6
                    else "inputs smaller than L2"},
-        "latency_ms": {"predict": round(pred_ms, 4), "attention": round(attn_ms, 4),
+        "latency_ms": {"predict": round(pred_ms, 4), "predict_pool": round(pool_ms, 4),
+                       "predict_select": round(sel_ms, 4), "attention": round(attn_ms, 4),
                        "step": round(ms_step, 4)},
+        "predict_roofline": {
+            "pool": {"bound": "hbm", "achieved": round(pbytes / (pool_ms * 1e-3) / 1e9, 1),
+                     "peak": hbm_peak, "unit": "GB/s",
+                     "frac": round(pbytes / (pool_ms * 1e-3) / 1e9 / hbm_peak, 4),
+                     "bytes_per_launch": pbytes,
+                     "kernel": "pool_kernel (+ k-bar and the K-code pass with INT8), "
+                               "algorithmic bytes / stage time"},
+            "select": {"bound": "fp32", "achieved": round(sel_flops / (sel_ms * 1e-3) / 1e12, 2),
+                       "peak": round(fp32_peak, 1), "unit": "TFLOP/s",
+                       "frac": round(sel_flops / (sel_ms * 1e-3) / 1e12 / fp32_peak, 4),
+                       "flops_per_launch": sel_flops,
+                       "kernel": "select_kernel: 2*d flops per visible (i, j) for S_hat; "
+                                 "peak = 148 SMs x 128 FP32 lanes x 2 x max SM clock"},
+        },
         "sparsity": sparsity,
         "work": {"tiles": tiles, "qk_blocks": qk_blocks, "pv_blocks": pv_blocks,
                  "pv_slices": pv_slices, "skipped_slices": skipped, "visible_blocks": vis},
@@ -313,6 +360,11 @@ def run_native(args, rank, world, local_rank):
                      "traffic": traffic,
                      "peak_source": f"{peak_src} bf16 sustained (MEASURED_PEAKS.json)",
                      "frac_of_burst_peak": round(achieved / peak_burst, 4),
+                     # INT8 Q K^T runs at twice the bf16 rate: the time the issued MMAs
+                     # need at the (sustained) peaks of their own dtypes, over the time taken
+                     "frac_mixed_peak": round(
+                         (qk_blocks * blk_flops / (2.0 if w.qk_int8 else 1.0)
+                          + pv_blocks * blk_flops) / (peak * 1e12) / (attn_ms * 1e-3), 4),
                      "kernel": "attn_kernel (tcgen05), issued MMA flops per launch / launch time"},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
@@ -338,6 +390,11 @@ def _gpu_uuid(torch, dev):
         return u if u.startswith("GPU-") else "GPU-" + u
     except Exception:
         return str(dev.index)
+
+
+def _visible_pairs(w):
+    """(query block, key block) pairs the select stage scores: causal-visible."""
+    return _visible_blocks(w)
 
 
 def _visible_blocks(w):

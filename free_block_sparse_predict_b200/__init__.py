@@ -24,7 +24,9 @@ __all__ = [
     "SpargeError", "SpargeParams", "SpargeStats", "make_params", "lib_path",
     "sparge_workspace_bytes", "sparge_hilbert_workspace_bytes", "sparge_hilbert_index",
     "sparge_hilbert_permute", "sparge_inverse_permute", "sparge_predict_mask",
-    "sparge_predict_mask_noalloc", "sparge_mask_compact", "sparge_attn_fwd", "sparge_device_status", "sparge_selftest_wait_timeout", "sparge_status_string",
+    "sparge_predict_pool", "sparge_predict_select", "sparge_predict_mask_noalloc",
+    "sparge_mask_compact", "sparge_attn_fwd", "sparge_device_status",
+    "sparge_selftest_wait_timeout", "sparge_status_string",
     "workspace", "predict_outputs", "sparge_forward",
 ]
 
@@ -99,6 +101,21 @@ def sparge_predict_mask(params, q, k, mask, kv_idx, kv_cnt, s_q, s_k, ws, stream
     _check(lib().sparge_predict_mask(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(mask),
                                      _ptr(kv_idx), _ptr(kv_cnt), _ptr(s_q), _ptr(s_k), _ptr(ws),
                                      ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def sparge_predict_pool(params, q, k, ws, stream=None) -> None:
+    """First half of sparge_predict_mask: block means, self-similarities and
+    (qk_int8) the INT8 codes, written into ws."""
+    _check(lib().sparge_predict_pool(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(ws),
+                                     ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def sparge_predict_select(params, mask, kv_idx, kv_cnt, s_q, s_k, ws, stream=None) -> None:
+    """Second half: the block mask and skip list from what sparge_predict_pool
+    left in the same ws."""
+    _check(lib().sparge_predict_select(ctypes.byref(params), _ptr(mask), _ptr(kv_idx),
+                                       _ptr(kv_cnt), _ptr(s_q), _ptr(s_k), _ptr(ws),
+                                       ws.numel() * ws.element_size(), _stream(stream)))
 
 
 def sparge_predict_mask_noalloc(params, q, k, mask, kv_idx, kv_cnt, s_q=None, s_k=None,

@@ -45,6 +45,8 @@ SIGNATURES = {
     "sparge_inverse_permute": (ctypes.c_int, [_V, _V, _I, _I, _I, _I, ctypes.c_int, _V, _V]),
     "sparge_predict_mask": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V, _V, _V, _S, _V]),
     "sparge_predict_mask_noalloc": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V, _V, _V]),
+    "sparge_predict_pool": (ctypes.c_int, [_P, _V, _V, _V, _S, _V]),
+    "sparge_predict_select": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V, _S, _V]),
     "sparge_mask_compact": (ctypes.c_int, [_P, _V, _V, _V, _V]),
     "sparge_attn_fwd": (ctypes.c_int, [_P, _V, _V, _V, _V, _V, _V, _V, _S, _V, _V]),
     "sparge_device_status": (ctypes.c_int, [_V, _V]),

@@ -5,7 +5,8 @@
 //
 // One CTA per 128-row query tile (b, h, i), 192 threads:
 //   warp 0     TMA producer: Q tile once, then K_j / V_j of the tile's skip
-//              list into a ring of shared-memory stages (128B swizzle).
+//              list into rings of shared-memory stages (128B swizzle), K
+//              running ahead of V.
 //   warp 1     allocates tensor memory; one thread issues every tcgen05.mma:
 //              S_t = Q K_t^T into a double-buffered S (TMEM), and
 //              O += P~_t V_t with P~ read from TMEM (aliased over S_t).
@@ -14,7 +15,7 @@
 //              rows (Eq. 3), P~ in fp16 back into TMEM, the row sum l, and a
 //              lazy rescale of its O row when the max grows by > 2^8.  The
 //              epilogue divides by l and stores O.
-// Pairs of CTAs share an SM (<= 97 KB shared memory, 256 TMEM columns each),
+// Pairs of CTAs share an SM (<= 113 KB shared memory, 256 TMEM columns each),
 // so one CTA's softmax overlaps the other's tensor-core work.
 //
 // Every mbarrier wait is bounded; a timeout sets the workspace status word to
@@ -51,13 +52,19 @@ struct Cfg {
   static constexpr int Q_BYTES = kBQ * D * QK_ES;
   static constexpr int K_BYTES = kBK * D * QK_ES;
   static constexpr int V_BYTES = kBK * D * 2;
-  static constexpr int STAGES = (D == 64) ? 4 : (MODE == kI8 ? 3 : 2);
+  // K_t is needed by S_t one block before V_t is needed by P~_t V_t, so K may
+  // run further ahead where shared memory allows (16-bit d = 128: 2 + 2
+  // stages; a third K stage there measured no faster).
+  static constexpr int K_STAGES = (D == 64) ? 6 : (MODE == kI8 ? 4 : 2);
+  static constexpr int V_STAGES = (D == 64) ? 4 : (MODE == kI8 ? 3 : 2);
   static constexpr int KSTEP = MODE == kI8 ? 32 : 16;         // MMA K per instruction
   static constexpr int QK_STEPS = D / KSTEP;
   static constexpr int TMEM_COLS = 256;                       // S0 | S1 | O
   static constexpr int O_COL = 128;
-  static constexpr int SMEM_TILES = Q_BYTES + STAGES * (K_BYTES + V_BYTES);
-  static constexpr int SMEM_BYTES = SMEM_TILES + 1024 /*align*/ + 512 /*barriers*/;
+  static constexpr int SMEM_TILES = Q_BYTES + K_STAGES * K_BYTES + V_STAGES * V_BYTES;
+  static constexpr int SMEM_BYTES = SMEM_TILES + 256 /*barriers*/;
+  // two CTAs per SM: 228 KB of shared memory, 1 KB of it reserved per CTA
+  static_assert(2 * (SMEM_BYTES + 1024) <= 228 * 1024, "two CTAs per SM");
 };
 
 struct AttnParams {
@@ -78,7 +85,7 @@ struct AttnParams {
 
 struct Bars {
   uint64_t q_full;
-  uint64_t k_full[4], k_empty[4], v_full[4], v_empty[4];
+  uint64_t k_full[6], k_empty[6], v_full[4], v_empty[4];
   uint64_t s_full[2], p_full[2];
   uint64_t o_done, o_final;
   uint32_t skip[2];  // byte q = 1 when softmax warp of quadrant q skips P~V
@@ -86,30 +93,17 @@ struct Bars {
   int abort;
 };
 
+static_assert(sizeof(Bars) <= 256, "barrier block");
+
 __device__ __forceinline__ void report_timeout(int32_t* status, volatile int* abort) {
   *abort = 1;
   atomicExch(status, int32_t(SPARGE_ETIMEOUT));
 }
 
-// ---- packed float32 pairs (sm_100a f32x2 arithmetic)
-__device__ __forceinline__ uint64_t pack2(float a, float b) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
-  return r;
-}
-__device__ __forceinline__ void unpack2(uint64_t v, float& a, float& b) {
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-}
-__device__ __forceinline__ uint64_t fma2(uint64_t a, uint64_t b, uint64_t c) {
-  uint64_t r;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
-  return r;
-}
-__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
-  uint64_t r;
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
-  return r;
-}
+// Whether a quarter of the exponentials run on the FMA pipe (exp2_poly2)
+// instead of the MUFU.  Off: once the INT8 scores stopped using the
+// conversion unit (which shares the MUFU pipe), all-MUFU measured 2-3% faster.
+constexpr bool kExp2OnFma = false;
 
 // 2^y for y <= 8 on the FMA pipe, for two values at once.  y = n + f with
 // n = round(y) (adding and subtracting 1.5 * 2^23) and f in [-1/2, 1/2];
@@ -137,16 +131,42 @@ __device__ __forceinline__ void exp2_poly2(float y0, float y1, float& r0, float&
   r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
 }
 
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// max of 64 floats (given as bits) by a depth-4 tree of three-input maxima
+__device__ __forceinline__ float max64(const uint32_t (&v)[64]) {
+  float a[22], b[8];
+#pragma unroll
+  for (int c = 0; c < 21; ++c)
+    a[c] = fmax3(__uint_as_float(v[3 * c]), __uint_as_float(v[3 * c + 1]),
+                 __uint_as_float(v[3 * c + 2]));
+  a[21] = __uint_as_float(v[63]);
+#pragma unroll
+  for (int c = 0; c < 7; ++c) b[c] = fmax3(a[3 * c], a[3 * c + 1], a[3 * c + 2]);
+  b[7] = a[21];
+  return fmax3(fmax3(b[0], b[1], b[2]), fmax3(b[3], b[4], b[5]), fmaxf(b[6], b[7]));
+}
+
 template <int D, int MODE>
 __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const __grid_constant__ AttnParams P) {
   using C = Cfg<D, MODE>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  // 128-byte-swizzled tiles need 1024-byte alignment; the dynamic shared
+  // memory of a kernel without static shared memory starts there.  Checked,
+  // not assumed: a misplaced window reports SPARGE_EUNSUPPORTED.
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_u32(smem_raw) & 1023u) {
+    if (threadIdx.x == 0) atomicCAS(P.status, 0, int32_t(SPARGE_EUNSUPPORTED));
+    return;
+  }
+  uint8_t* smem = smem_raw;
   uint8_t* sQ = smem;
   uint8_t* sK = sQ + C::Q_BYTES;
-  uint8_t* sV = sK + C::STAGES * C::K_BYTES;
-  Bars* bars = reinterpret_cast<Bars*>(sV + C::STAGES * C::V_BYTES);
+  uint8_t* sV = sK + C::K_STAGES * C::K_BYTES;
+  Bars* bars = reinterpret_cast<Bars*>(sV + C::V_STAGES * C::V_BYTES);
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -166,9 +186,11 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const __grid_constant
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < C::STAGES; ++s) {
+    for (int s = 0; s < C::K_STAGES; ++s) {
       mbar_init(&bars->k_full[s], 1);
       mbar_init(&bars->k_empty[s], 1);
+    }
+    for (int s = 0; s < C::V_STAGES; ++s) {
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->v_empty[s], 1);
     }
@@ -198,36 +220,52 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const __grid_constant
       tma_prefetch_desc(&P.tmQ);
       tma_prefetch_desc(&P.tmK);
       tma_prefetch_desc(&P.tmV);
-      int k_issued[4] = {0, 0, 0, 0}, v_issued[4] = {0, 0, 0, 0};
+      int k_issued[C::K_STAGES] = {}, v_issued[C::V_STAGES] = {};
       mbar_expect_tx(&bars->q_full, C::Q_BYTES);
       for (int x = 0; x < C::QK_BOXES; ++x)
         tma_load_3d(sQ + x * (kBQ * 128), &P.tmQ, &bars->q_full, x * C::BOX_X, i * kBQ,
                     int32_t(bh));
-      bool ok = true;
-      for (int t = 0; t < n && ok; ++t) {
-        const int st = t % C::STAGES;
-        const int use = t / C::STAGES;
+      // K_t into stage t % K_STAGES once Q K_{t-K_STAGES}^T has read it
+      auto load_k = [&](int t) -> bool {
+        const int st = t % C::K_STAGES, use = t / C::K_STAGES;
+        if (use > 0 && !mbar_wait(&bars->k_empty[st], (use - 1) & 1, abort, P.status)) return false;
         const int j = __ldg(kv_list + t);
-        if (use > 0 && !(ok = mbar_wait(&bars->k_empty[st], (use - 1) & 1, abort, P.status))) break;
         mbar_expect_tx(&bars->k_full[st], C::K_BYTES);
         for (int x = 0; x < C::QK_BOXES; ++x)
           tma_load_3d(sK + st * C::K_BYTES + x * (kBK * 128), &P.tmK, &bars->k_full[st],
                       x * C::BOX_X, j * kBK, int32_t(bhk));
         ++k_issued[st];
-        if (use > 0 && !(ok = mbar_wait(&bars->v_empty[st], (use - 1) & 1, abort, P.status))) break;
+        return true;
+      };
+      // V_t once P~_{t-V_STAGES} V_{t-V_STAGES} has read its stage
+      auto load_v = [&](int t) -> bool {
+        const int st = t % C::V_STAGES, use = t / C::V_STAGES;
+        if (use > 0 && !mbar_wait(&bars->v_empty[st], (use - 1) & 1, abort, P.status)) return false;
+        const int j = __ldg(kv_list + t);
         mbar_expect_tx(&bars->v_full[st], C::V_BYTES);
         for (int x = 0; x < C::V_BOXES; ++x)
           tma_load_3d(sV + st * C::V_BYTES + x * (kBK * 128), &P.tmV, &bars->v_full[st], x * 64,
                       j * kBK, int32_t(bhk));
         ++v_issued[st];
+        return true;
+      };
+      // K runs K_STAGES blocks ahead of V: the tensor pipe needs K_{t+1} (for
+      // S_{t+1}) before V_t (for P~_t V_t).  V_t waits for P~V of block
+      // t - V_STAGES, which the tensor pipe runs before S_t, whose end frees
+      // the stage of K_{t+K_STAGES}: so a V wait never holds K back.
+      bool ok = true;
+      for (int t = 0; t < n && t < C::K_STAGES && ok; ++t) ok = load_k(t);
+      for (int t = 0; t < n && ok; ++t) {
+        ok = load_v(t);
+        if (ok && t + C::K_STAGES < n) ok = load_k(t + C::K_STAGES);
       }
       if (!ok) report_timeout(P.status, abort);
       // let every copy this thread started land before the CTA can exit
       mbar_wait_teardown(&bars->q_full, 0);
-      for (int s = 0; s < C::STAGES; ++s) {
+      for (int s = 0; s < C::K_STAGES; ++s)
         if (k_issued[s] > 0) mbar_wait_teardown(&bars->k_full[s], (k_issued[s] - 1) & 1);
+      for (int s = 0; s < C::V_STAGES; ++s)
         if (v_issued[s] > 0) mbar_wait_teardown(&bars->v_full[s], (v_issued[s] - 1) & 1);
-      }
     }
   } else if (warp == 1) {
     // =================================================== MMA issuer
@@ -244,8 +282,8 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const __grid_constant
         if (!mbar_wait(&bars->p_full[sb], (u >> 1) & 1, abort, P.status)) return false;
         tc_fence_after();
         const uint32_t flags = *reinterpret_cast<volatile uint32_t*>(&bars->skip[sb]);
-        const int stv = u % C::STAGES;
-        if (!mbar_wait(&bars->v_full[stv], (u / C::STAGES) & 1, abort, P.status)) return false;
+        const int stv = u % C::V_STAGES;
+        if (!mbar_wait(&bars->v_full[stv], (u / C::V_STAGES) & 1, abort, P.status)) return false;
         tc_fence_after();
         if (flags != 0x01010101u) {
           const uint32_t a_tmem = tmem + uint32_t(sb * kBK);
@@ -263,8 +301,8 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const __grid_constant
         return true;
       };
       for (int t = 0; t < n && ok; ++t) {
-        const int st = t % C::STAGES;
-        if (!(ok = mbar_wait(&bars->k_full[st], (t / C::STAGES) & 1, abort, P.status))) break;
+        const int st = t % C::K_STAGES;
+        if (!(ok = mbar_wait(&bars->k_full[st], (t / C::K_STAGES) & 1, abort, P.status))) break;
         tc_fence_after();
         const int sb = t & 1;
         const uint32_t kbase = sKa + uint32_t(st * C::K_BYTES);
@@ -325,7 +363,9 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const __grid_constant
       if (P.causal) lim = min(lim, row_g - key0 + 1);
       if (!row_ok || j < 0) lim = 0;
 
-      if (!(ok = mbar_wait(&bars->s_full[sb], (t >> 1) & 1, abort, P.status))) break;
+      // the outcome of every wait is made warp-uniform before it steers control
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[sb], (t >> 1) & 1, abort, P.status));
+      if (!ok) break;
       tc_fence_after();
       uint32_t raw[64];
       {
@@ -335,38 +375,26 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const __grid_constant
         tmem_ld32(lane_addr + uint32_t(sb * kBK + 32), r1);
         tmem_wait_ld();
       }
-      // row max on the raw accumulators (sc > 0 preserves the order), by a tree
-      float m_loc;
+      // INT8 scores become floats first, without the conversion unit (it
+      // shares the MUFU pipe with ex2): the bits of 1.5 * 2^23 + x are that
+      // float exactly for |x| < 2^22, and an INT8 score of d = 128 is at most
+      // 127^2 * 128; the order of x is kept, so the max runs on them as is.
+      constexpr float kMagic = 12582912.0f;
       if (MODE == kI8) {
-        if (lim < 64) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (c >= lim) raw[c] = 0x80000000u;
-        }
-        int a[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c) a[c] = max(int32_t(raw[c]), int32_t(raw[c + 32]));
-#pragma unroll
-        for (int w2 = 16; w2 > 0; w2 >>= 1)
-#pragma unroll
-          for (int c = 0; c < w2; ++c) a[c] = max(a[c], a[c + w2]);
-        m_loc = a[0] == INT32_MIN ? -INFINITY : float(a[0]) * sc;
-      } else {
-        if (lim < 64) {
-#pragma unroll
-          for (int c = 0; c < 64; ++c)
-            if (c >= lim) raw[c] = 0xFF800000u;  // -inf
-        }
-        float a[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-          a[c] = fmaxf(__uint_as_float(raw[c]), __uint_as_float(raw[c + 32]));
-#pragma unroll
-        for (int w2 = 16; w2 > 0; w2 >>= 1)
-#pragma unroll
-          for (int c = 0; c < w2; ++c) a[c] = fmaxf(a[c], a[c + w2]);
-        m_loc = a[0] * sc;
+        for (int c = 0; c < 64; ++c) raw[c] += 0x4B400000u;
       }
+      if (lim < 64) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (c >= lim) raw[c] = 0xFF800000u;  // -inf
+      }
+      // row max on the raw accumulators (sc > 0 preserves the order), by a
+      // tree of three-input maxima
+      const float m_raw = max64(raw);
+      // (an INT8 block scale can be 0: keep an all-masked row at -inf)
+      const float m_loc =
+          m_raw == -INFINITY ? -INFINITY : (MODE == kI8 ? m_raw - kMagic : m_raw) * sc;
       const float m_new = fmaxf(m_true, m_loc);
       const float diff = (m_loc == -INFINITY) ? -INFINITY : (m_loc - m_new);
       const bool skip = __all_sync(0xffffffffu, diff < P.lam2);
@@ -374,7 +402,8 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const __grid_constant
       const bool grow = m_new > m_sc + kRescaleThreshold;
       const bool need_o = grow && (m_sc != -INFINITY);
       if (__any_sync(0xffffffffu, need_o)) {
-        if (!(ok = mbar_wait(&bars->o_done, (t - 1) & 1, abort, P.status))) break;
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_done, (t - 1) & 1, abort, P.status));
+        if (!ok) break;
         tc_fence_after();
         const float alpha = need_o ? ex2_approx(m_sc - m_new) : 1.f;
 #pragma unroll 1
@@ -396,17 +425,11 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const __grid_constant
       float pv[64];
 #pragma unroll
       for (int c = 0; c < 64; c += 2) {
-        float x0, x1;
-        if (MODE == kI8) {
-          x0 = float(int32_t(raw[c]));
-          x1 = float(int32_t(raw[c + 1]));
-        } else {
-          x0 = __uint_as_float(raw[c]);
-          x1 = __uint_as_float(raw[c + 1]);
-        }
+        uint64_t x2 = pack2(__uint_as_float(raw[c]), __uint_as_float(raw[c + 1]));
+        if (MODE == kI8) x2 = add2(x2, pack2(-kMagic, -kMagic));  // exact
         float y0, y1;
-        unpack2(fma2(pack2(x0, x1), sc2, nb2), y0, y1);
-        if ((c & 7) == 6) {
+        unpack2(fma2(x2, sc2, nb2), y0, y1);
+        if (kExp2OnFma && (c & 7) == 6) {
           exp2_poly2(y0, y1, pv[c], pv[c + 1]);
         } else {
           pv[c] = ex2_approx(y0);
@@ -447,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const __grid_constant
     }
     if (!ok) report_timeout(P.status, abort);
     // ---- epilogue: O / l
-    if (ok && n > 0) ok = mbar_wait(&bars->o_final, 0, abort, P.status);
+    if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_final, 0, abort, P.status));
     if (!ok) report_timeout(P.status, abort);
     tc_fence_after();
     if (ok) {

@@ -1,13 +1,13 @@
 // Stage 1 of SpargeAttn: the sparse-block predictor (paper review page,
 // section 三, Eq. 4-9 and Algorithm 1 steps 2-5).
 //
-//   pool_warp_kernel<.., 0>  one pass over Q and K (HBM bound), one warp per
-//                   block: the mean token (Eq. 4, 5) and the self-similarity
+//   pool_kernel<.., 0>  one pass over Q and K (HBM bound), one warp per
+//                   64-row slab held in registers: the mean token (Eq. 4, 5) and the self-similarity
 //                   CosSim (Eq. 6, read as the mean of the block's token cosine
 //                   matrix), via mean_{a,b} xh_a.xh_b = |sum_a xh_a|^2 / n^2.
 //                   With INT8 it also quantises Q per block (Algorithm 1 step 2).
-//   kbar_kernel     per-head mean of K from the block means (K smoothing).
-//   pool_warp_kernel<.., 1>  per-block INT8 of K - kbar (second pass over K).
+//   kbar_*_kernel   per-head mean of K from the block means (K smoothing).
+//   pool_kernel<.., 1>  per-block INT8 of K - kbar (second pass over K).
 //   select_kernel   per query block: S_hat = scale q_i k^T with -inf columns
 //                   (Eq. 7), row softmax, TopCdf(tau) (Eq. 8) by an exact
 //                   value-threshold bisection, the fix-block rule (Eq. 9), and
@@ -25,39 +25,10 @@
 namespace sparge {
 namespace {
 
-constexpr int kPoolThreads = 256;
-
-__device__ __forceinline__ void unpack8(const uint4& raw, float (&x)[8], bool bf16) {
-  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    if (bf16) {
-      x[2 * i] = __uint_as_float(w[i] << 16);
-      x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    } else {
-      __half2 h = *reinterpret_cast<const __half2*>(&w[i]);
-      float2 f = __half22float2(h);
-      x[2 * i] = f.x;
-      x[2 * i + 1] = f.y;
-    }
-  }
-}
-
-// code = rint(x * inv), inv = 127 / absmax of the block, clamped to +-127
-__device__ __forceinline__ int8_t quant1(float x, float inv) {
-  float v = rintf(__fmul_rn(x, inv));
-  v = fminf(127.f, fmaxf(-127.f, v));
-  return static_cast<int8_t>(v);
-}
-
-__device__ __forceinline__ uint2 pack_codes(const float (&x)[8], float inv) {
-  uint32_t lo = 0, hi = 0;
-#pragma unroll
-  for (int e = 0; e < 4; ++e) lo |= (uint32_t)(uint8_t)quant1(x[e], inv) << (8 * e);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) hi |= (uint32_t)(uint8_t)quant1(x[4 + e], inv) << (8 * e);
-  return make_uint2(lo, hi);
-}
+constexpr int kPoolThreads = 128;
+constexpr int kPoolMinBlocks = 4;  // <= 128 registers; a slab's rows take 64 of them
+constexpr int kPoolBQ = 128;       // query block rows (the only b_q the library accepts)
+constexpr int kPoolBK = 64;        // key block rows
 
 struct PoolArgs {
   const void* q;
@@ -85,77 +56,208 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
   return r;
 }
 
-// One warp per block, no shared memory and no CTA barrier: lane (ro, c) owns
-// the 16-byte chunk c of rows ro, ro + RPW, ...  Row norms reduce over the CH
-// lanes of a row, column sums over the RPW row groups at the end.
+// Same bits, but opaque to the compiler: keeps it from holding every row's
+// unpacked floats live between two passes over the registers (it would
+// otherwise reuse the first unpacking and spill).
+__device__ __forceinline__ uint4 opaque(uint4 v) {
+  asm volatile("" : "+r"(v.x), "+r"(v.y), "+r"(v.z), "+r"(v.w));
+  return v;
+}
+
+__device__ __forceinline__ void named_barrier(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// The two 16-bit values of w as a packed fp32 pair (exact).
+template <bool BF16>
+__device__ __forceinline__ uint64_t widen2(uint32_t w) {
+  if (BF16) return pack2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&w));
+  return pack2(f.x, f.y);
+}
+
+// Per-half running max of |x| on packed 16-bit values: max.xorsign.abs keeps
+// the larger magnitude (its sign bit is dropped at the end).  Exact.
+template <bool BF16>
+__device__ __forceinline__ uint32_t absmax2(uint32_t acc, uint32_t w) {
+  uint32_t r;
+  if (BF16)
+    asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(acc), "r"(w));
+  else
+    asm("max.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(r) : "r"(acc), "r"(w));
+  return r;
+}
+
+template <bool BF16>
+__device__ __forceinline__ float absmax2_value(uint32_t acc) {
+  const uint32_t m = acc & 0x7FFF7FFFu;
+  if (BF16) return fmaxf(__uint_as_float(m << 16), __uint_as_float(m & 0xFFFF0000u));
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&m));
+  return fmaxf(f.x, f.y);
+}
+
+// Eight INT8 codes rint(x * inv) of a packed fp32 row chunk.  q = x * inv is
+// the IEEE-rounded fp32 product (__fmul_rn), then q + 1.5 * 2^23 (__fadd_rn)
+// rounds q to the nearest integer, ties to even, exactly as rint does for
+// |q| < 2^22; |q| <= 127 (x is bounded by the absmax that inv comes from), so
+// the code is the low byte of that sum's bits, two's complement included.
+// Scalar on purpose: with the packed f32x2 forms the compiler fused the
+// product into the add, rounding the exact product instead of q, which turns
+// ties such as q = 63.5 (from a product just below it) the other way.
+__device__ __forceinline__ uint2 codes8(const uint64_t (&x2)[4], float inv) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  uint32_t bits[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float a, b;
+    unpack2(x2[i], a, b);
+    bits[2 * i] = __float_as_uint(__fadd_rn(__fmul_rn(a, inv), kMagic));
+    bits[2 * i + 1] = __float_as_uint(__fadd_rn(__fmul_rn(b, inv), kMagic));
+  }
+  const uint32_t lo = __byte_perm(__byte_perm(bits[0], bits[1], 0x0040),
+                                  __byte_perm(bits[2], bits[3], 0x0040), 0x5410);
+  const uint32_t hi = __byte_perm(__byte_perm(bits[4], bits[5], 0x0040),
+                                  __byte_perm(bits[6], bits[7], 0x0040), 0x5410);
+  return make_uint2(lo, hi);
+}
+
+// One warp per SLAB-row slab of a block, held in registers for the whole
+// pass, so every byte of Q and K is read from HBM exactly once per pass.
+// Lane (ro, c) owns the 16-byte chunk c of rows ro, ro + RPW, ...  Arithmetic
+// runs on packed fp32 pairs; the squared row norms of a lane's NR rows are
+// reduced over the CH lanes of each row by a transposing butterfly (each step
+// halves the rows a lane carries), and the inverse norms broadcast back.  The
+// G = block rows / SLAB warps of one block are adjacent in the CTA and combine
+// their partial sums and absmax through shared memory (one named barrier),
+// always in slab order, so the result does not depend on scheduling.
 //   KIND 0  pooling pass over Q blocks then K blocks: mean token, CosSim by
 //           |sum xhat|^2 / n^2, and with q_codes the INT8 codes of Q.
 //   KIND 1  INT8 pass over K blocks: codes of K - kbar and their scales.
-// The codes are a second, L2-resident read of the block once its absmax is
-// known: code = rint(x * (127 / absmax)), clamped to +-127.
-template <int D, bool BF16, int KIND>
-__global__ void __launch_bounds__(256) pool_warp_kernel(PoolArgs a) {
-  constexpr int CH = D * 2 / 16;          // lanes per row
-  constexpr int RPW = 32 / CH;            // rows per warp pass
-  constexpr int UNROLL = 4;
-  const int lane = threadIdx.x & 31;
-  const int64_t id0 = int64_t(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (id0 >= a.nblocks) return;
-  int64_t id = id0;
-  const bool isQ = KIND == 0 && id < a.nQblocks;
-  if (KIND == 0 && !isQ) id -= a.nQblocks;
-  const int T = isQ ? a.Tm : a.Tn;
-  const int BLK = isQ ? a.bq : a.bk;
-  const int64_t bh = id / T;
-  const int blk = int(id % T);
-  const int rows = min(BLK, a.N - blk * BLK);
-  const uint16_t* src = static_cast<const uint16_t*>(isQ ? a.q : a.k) +
-                        (bh * a.N + int64_t(blk) * BLK) * D;
-  const int c = lane % CH, ro = lane / CH;
+template <int D, bool BF16, int KIND, int SLAB>
+__global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(PoolArgs a) {
+  constexpr int CH = D * 2 / 16;  // lanes per row
+  constexpr int RPW = 32 / CH;    // rows per warp-wide load
+  constexpr int NR = SLAB / RPW;  // rows per lane
+  constexpr int R = NR / CH;      // rows whose norm a lane holds after the butterfly
+  constexpr int WARPS = kPoolThreads / 32;
+  constexpr int GQ = kPoolBQ / SLAB, GK = kPoolBK / SLAB;
+  static_assert(WARPS % GQ == 0 && GQ % GK == 0, "groups must tile the CTA");
+  static_assert(NR % CH == 0, "butterfly needs NR a multiple of CH");
+  __shared__ float part[WARPS][2 * D];
+  __shared__ float pmax[WARPS];
 
-  float kb[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t gw = int64_t(blockIdx.x) * WARPS + warp;
+  const int64_t nQw = a.nQblocks * GQ;
+  const bool isQ = KIND == 0 && gw < nQw;
+  const int G = isQ ? GQ : GK;
+  const int64_t rel = isQ ? gw : gw - nQw;
+  const int64_t blkid = rel / G;
+  const int sub = int(rel % G);  // slab index inside the block
+  if (blkid >= (isQ ? a.nQblocks : a.nblocks - a.nQblocks)) return;  // whole groups leave
+  const int T = isQ ? a.Tm : a.Tn;
+  const int BLK = isQ ? kPoolBQ : kPoolBK;
+  const int64_t bh = blkid / T;
+  const int blk = int(blkid % T);
+  const int rows = min(BLK, a.N - blk * BLK);
+  const int srows = max(0, min(SLAB, rows - sub * SLAB));
+  const int c = lane % CH, ro = lane / CH;
+  const int64_t row0 = bh * a.N + int64_t(blk) * BLK + sub * SLAB;
+  const uint16_t* src = static_cast<const uint16_t*>(isQ ? a.q : a.k) + row0 * D + c * 8;
+
+  uint4 raw[NR];
+#pragma unroll
+  for (int u = 0; u < NR; ++u) {
+    const int r = ro + u * RPW;
+    raw[u] = r < srows ? ld_stream(src + int64_t(r) * D) : make_uint4(0, 0, 0, 0);
+  }
+  uint64_t nkb2[4];  // -kbar of this lane's 8 columns, as pairs
   if (KIND == 1) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) kb[e] = a.kbar[bh * D + c * 8 + e];
+    for (int e = 0; e < 4; ++e)
+      nkb2[e] = pack2(-a.kbar[bh * D + c * 8 + 2 * e], -a.kbar[bh * D + c * 8 + 2 * e + 1]);
   }
+
   float sx[8], su[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) sx[e] = su[e] = 0.f;
   float amax = 0.f;
-  for (int r0 = ro; r0 < BLK; r0 += RPW * UNROLL) {
-    uint4 raw[UNROLL];
+  if (KIND == 0) {
+    // ---- squared row norms, one value per row
+    float v[NR];
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      const int r = r0 + u * RPW;
-      raw[u] = r < rows ? ld_stream(src + int64_t(r) * D + c * 8) : make_uint4(0, 0, 0, 0);
+    for (int u = 0; u < NR; ++u) {
+      const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
+      uint64_t acc = pack2(0.f, 0.f);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint64_t x2 = widen2<BF16>(w[e]);
+        acc = fma2(x2, x2, acc);
+      }
+      float s0, s1;
+      unpack2(acc, s0, s1);
+      v[u] = s0 + s1;
+    }
+    // ---- butterfly over the CH lanes of a row: at offset o the lanes with
+    // bit o set keep the upper half of their rows and send the lower half
+#pragma unroll
+    for (int o = CH / 2, cnt = NR; o > 0; o >>= 1, cnt >>= 1) {
+      const bool up = (lane & o) != 0;
+#pragma unroll
+      for (int k = 0; k < cnt / 2; ++k) {
+        const float send = up ? v[k] : v[k + cnt / 2];
+        const float keep = up ? v[k + cnt / 2] : v[k];
+        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
+    }
+    // lane c of a row group now holds rows c * R .. c * R + R - 1
+    float inv_own[R];
+#pragma unroll
+    for (int t = 0; t < R; ++t) inv_own[t] = v[t] > 0.f ? rsqrtf(v[t]) : 0.f;
+    const int group_base = lane & ~(CH - 1);
+    // ---- column sums of x and of x / |x_row|, and the exact |x| max
+    uint64_t sx2[4], su2[4];
+    uint32_t am2[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sx2[e] = su2[e] = pack2(0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < NR; ++u) {
+      const float inv = __shfl_sync(0xffffffffu, inv_own[u % R], group_base | (u / R));
+      const uint64_t iv2 = pack2(inv, inv);
+      const uint4 rw = opaque(raw[u]);
+      const uint32_t w[4] = {rw.x, rw.y, rw.z, rw.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint64_t x2 = widen2<BF16>(w[e]);
+        sx2[e] = add2(sx2[e], x2);
+        su2[e] = fma2(x2, iv2, su2[e]);
+        am2[e] = absmax2<BF16>(am2[e], w[e]);
+      }
     }
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      const bool valid = r0 + u * RPW < rows;
-      float x[8];
-      unpack8(raw[u], x, BF16);
-      if (KIND == 0) {
-        float ss = 0.f;
+    for (int e = 0; e < 4; ++e) {
+      unpack2(sx2[e], sx[2 * e], sx[2 * e + 1]);
+      unpack2(su2[e], su[2 * e], su[2 * e + 1]);
+    }
+    amax = absmax2_value<BF16>(absmax2<BF16>(absmax2<BF16>(am2[0], am2[1]),
+                                             absmax2<BF16>(am2[2], am2[3])));
+  } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ss = fmaf(x[e], x[e], ss);
+    for (int u = 0; u < NR; ++u) {
+      if (ro + u * RPW < srows) {
+        const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
 #pragma unroll
-        for (int o = CH / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-        const float inv = ss > 0.f ? 1.0f / sqrtf(ss) : 0.f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          sx[e] += x[e];
-          su[e] = fmaf(x[e], inv, su[e]);
-          amax = fmaxf(amax, fabsf(x[e]));
+        for (int e = 0; e < 4; ++e) {
+          float d0, d1;
+          unpack2(add2(widen2<BF16>(w[e]), nkb2[e]), d0, d1);
+          amax = fmaxf(amax, fmaxf(fabsf(d0), fabsf(d1)));
         }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          if (valid) amax = fmaxf(amax, fabsf(__fsub_rn(x[e], kb[e])));
       }
     }
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   if (KIND == 0) {
-    // column sums over the RPW row groups
 #pragma unroll
     for (int o = CH; o < 32; o <<= 1)
 #pragma unroll
@@ -163,6 +265,35 @@ __global__ void __launch_bounds__(256) pool_warp_kernel(PoolArgs a) {
         sx[e] += __shfl_xor_sync(0xffffffffu, sx[e], o);
         su[e] += __shfl_xor_sync(0xffffffffu, su[e], o);
       }
+  }
+  if (G > 1) {
+    if (KIND == 0 && ro == 0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        part[warp][c * 8 + e] = sx[e];
+        part[warp][D + c * 8 + e] = su[e];
+      }
+    }
+    if (lane == 0) pmax[warp] = amax;
+    named_barrier(1 + warp / G, 32 * G);
+    const int w0 = warp - sub;
+    if (KIND == 0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        sx[e] = part[w0][c * 8 + e];
+        su[e] = part[w0][D + c * 8 + e];
+      }
+      for (int g = 1; g < G; ++g)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          sx[e] += part[w0 + g][c * 8 + e];
+          su[e] += part[w0 + g][D + c * 8 + e];
+        }
+    }
+    amax = pmax[w0];
+    for (int g = 1; g < G; ++g) amax = fmaxf(amax, pmax[w0 + g]);
+  }
+  if (KIND == 0 && sub == 0) {
     float uu = 0.f;
 #pragma unroll
     for (int e = 0; e < 8; ++e) uu = fmaf(su[e], su[e], uu);
@@ -179,57 +310,52 @@ __global__ void __launch_bounds__(256) pool_warp_kernel(PoolArgs a) {
   }
   const bool quantise = KIND == 1 || (isQ && a.q_codes != nullptr);
   if (!quantise) return;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  const float delta = amax / 127.0f;
   const float inv = amax > 0.f ? 127.0f / amax : 0.f;
-  if (lane == 0) (KIND == 1 ? a.dk : a.dq)[bh * T + blk] = delta;
-  int8_t* codes = (KIND == 1 ? a.k_codes : a.q_codes) + (bh * a.N + int64_t(blk) * BLK) * D;
-  for (int r0 = ro; r0 < rows; r0 += RPW * UNROLL) {
-    uint4 raw[UNROLL];
+  if (sub == 0 && lane == 0) (KIND == 1 ? a.dk : a.dq)[bh * T + blk] = amax / 127.0f;
+  int8_t* codes = (KIND == 1 ? a.k_codes : a.q_codes) + row0 * D + c * 8;
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      const int r = r0 + u * RPW;
-      raw[u] = r < rows ? *reinterpret_cast<const uint4*>(src + int64_t(r) * D + c * 8)
-                        : make_uint4(0, 0, 0, 0);
-    }
+  for (int u = 0; u < NR; ++u) {
+    const int r = ro + u * RPW;
+    if (r < srows) {
+      const uint4 rw = opaque(raw[u]);
+      const uint32_t w[4] = {rw.x, rw.y, rw.z, rw.w};
+      uint64_t x2[4];
 #pragma unroll
-    for (int u = 0; u < UNROLL; ++u) {
-      const int r = r0 + u * RPW;
-      if (r < rows) {
-        float x[8];
-        unpack8(raw[u], x, BF16);
-        if (KIND == 1) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], kb[e]);
-        }
-        *reinterpret_cast<uint2*>(codes + int64_t(r) * D + c * 8) = pack_codes(x, inv);
+      for (int e = 0; e < 4; ++e) {
+        x2[e] = widen2<BF16>(w[e]);
+        if (KIND == 1) x2[e] = add2(x2[e], nkb2[e]);
       }
+      *reinterpret_cast<uint2*>(codes + int64_t(r) * D) = codes8(x2, inv);
     }
   }
 }
 
-// kbar[bh, :] = (sum_j n_j * k_mean[bh, j, :]) / N, a fixed-order two-level sum
+// kbar[bh, :] = (sum_j n_j * k_mean[bh, j, :]) / N in a fixed order: slice s
+// of kKbarSlices sums its key blocks into part[bh, s, :], then one CTA per head
+// adds the slices in index order.
 template <int D>
-__global__ void __launch_bounds__(1024) kbar_kernel(const float* k_mean, float* kbar, int32_t N,
-                                                    int32_t bk, int32_t Tn) {
-  constexpr int G = 1024 / D;
-  __shared__ float part[G][D];
-  const int64_t bh = blockIdx.x;
-  const int g = threadIdx.x / D, col = threadIdx.x % D;
+__global__ void __launch_bounds__(D) kbar_partial_kernel(const float* k_mean, float* part,
+                                                         int32_t N, int32_t bk, int32_t Tn) {
+  const int64_t bh = blockIdx.x / kKbarSlices;
+  const int sl = int(blockIdx.x % kKbarSlices), col = threadIdx.x;
+  const int per = (Tn + kKbarSlices - 1) / kKbarSlices;
+  const int j0 = sl * per, j1 = min(Tn, j0 + per);
   float acc = 0.f;
-  for (int j = g; j < Tn; j += G) {
+  for (int j = j0; j < j1; ++j) {
     const int n = min(bk, N - j * bk);
     acc = fmaf(k_mean[(bh * Tn + j) * D + col], float(n), acc);
   }
-  part[g][col] = acc;
-  __syncthreads();
-  if (g == 0) {
-    float s = 0.f;
-#pragma unroll
-    for (int i = 0; i < G; ++i) s += part[i][col];
-    kbar[bh * D + col] = s / float(N);
-  }
+  part[(bh * kKbarSlices + sl) * D + col] = acc;
+}
+
+template <int D>
+__global__ void __launch_bounds__(D) kbar_final_kernel(const float* part, float* kbar, int32_t N) {
+  const int64_t bh = blockIdx.x;
+  const int col = threadIdx.x;
+  float s = 0.f;
+#pragma unroll 8
+  for (int sl = 0; sl < kKbarSlices; ++sl) s += part[(bh * kKbarSlices + sl) * D + col];
+  kbar[bh * D + col] = s / float(N);
 }
 
 // ------------------------------------------------------------------ select
@@ -280,38 +406,59 @@ __global__ void __launch_bounds__(256) select_kernel(SelectArgs a) {
     const int r = idx / D, e = idx % D;
     qs[idx] = (i0 + r < a.Tm) ? a.q_mean[(bh * a.Tm + i0 + r) * D + e] : 0.f;
   }
-  // ---- S_hat rows i0..i0+7 against every visible key block (Eq. 7, before masking)
-  for (int jt = 0; jt * kSelCols < jcount; ++jt) {
-    float acc[kSelRows];
+  // ---- S_hat rows i0..i0+7 against every visible key block (Eq. 7, before
+  // masking).  The key means stream through shared memory in chunks of
+  // kSelCols blocks x 32 columns; each thread prefetches its share of the
+  // next chunk into registers while the current one is multiplied, so the
+  // L2 latency of the loads overlaps the arithmetic.
+  const int njt = (jcount + kSelCols - 1) / kSelCols;
+  const int nchunks = njt * (D / 32);
+  float4 pre[kSelCols * 8 / 256];
+  auto fetch = [&](int chunk) {
+    const int jt = chunk / (D / 32), ec = (chunk % (D / 32)) * 32;
 #pragma unroll
-    for (int r = 0; r < kSelRows; ++r) acc[r] = 0.f;
-    for (int ec = 0; ec < D; ec += 32) {
-      __syncthreads();
-      for (int idx = tid; idx < kSelCols * 8; idx += 256) {
-        const int jl = idx >> 3, f4 = idx & 7, j = jt * kSelCols + jl;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (j < jcount)
-          v = *reinterpret_cast<const float4*>(a.k_mean + (kbh * a.Tn + j) * D + ec + f4 * 4);
-        *reinterpret_cast<float4*>(ks + jl * kKPad + f4 * 4) = v;
-      }
-      __syncthreads();
+    for (int u = 0; u < kSelCols * 8 / 256; ++u) {
+      const int idx = tid + u * 256;
+      const int jl = idx >> 3, f4 = idx & 7, j = jt * kSelCols + jl;
+      pre[u] = j < jcount
+                   ? *reinterpret_cast<const float4*>(a.k_mean + (kbh * a.Tn + j) * D + ec + f4 * 4)
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  };
+  if (nchunks > 0) fetch(0);
+  float acc[kSelRows];
 #pragma unroll
-      for (int e = 0; e < 32; e += 4) {
-        const float4 kv = *reinterpret_cast<const float4*>(ks + tid * kKPad + e);
+  for (int r = 0; r < kSelRows; ++r) acc[r] = 0.f;
+  for (int chunk = 0; chunk < nchunks; ++chunk) {
+    const int jt = chunk / (D / 32), ec = (chunk % (D / 32)) * 32;
+    __syncthreads();  // the previous chunk is no longer read
 #pragma unroll
-        for (int r = 0; r < kSelRows; ++r) {
-          const float4 qv = *reinterpret_cast<const float4*>(qs + r * D + ec + e);
-          acc[r] = fmaf(qv.x, kv.x, acc[r]);
-          acc[r] = fmaf(qv.y, kv.y, acc[r]);
-          acc[r] = fmaf(qv.z, kv.z, acc[r]);
-          acc[r] = fmaf(qv.w, kv.w, acc[r]);
-        }
+    for (int u = 0; u < kSelCols * 8 / 256; ++u) {
+      const int idx = tid + u * 256;
+      *reinterpret_cast<float4*>(ks + (idx >> 3) * kKPad + (idx & 7) * 4) = pre[u];
+    }
+    __syncthreads();
+    if (chunk + 1 < nchunks) fetch(chunk + 1);
+#pragma unroll
+    for (int e = 0; e < 32; e += 4) {
+      const float4 kv = *reinterpret_cast<const float4*>(ks + tid * kKPad + e);
+#pragma unroll
+      for (int r = 0; r < kSelRows; ++r) {
+        const float4 qv = *reinterpret_cast<const float4*>(qs + r * D + ec + e);
+        acc[r] = fmaf(qv.x, kv.x, acc[r]);
+        acc[r] = fmaf(qv.y, kv.y, acc[r]);
+        acc[r] = fmaf(qv.z, kv.z, acc[r]);
+        acc[r] = fmaf(qv.w, kv.w, acc[r]);
       }
     }
-    const int j = jt * kSelCols + tid;
-    if (j < jcount) {
+    if (ec + 32 == D) {
+      const int j = jt * kSelCols + tid;
+      if (j < jcount) {
 #pragma unroll
-      for (int r = 0; r < kSelRows; ++r) shat[r * a.Tn + j] = acc[r] * a.scale;
+        for (int r = 0; r < kSelRows; ++r) shat[r * a.Tn + j] = acc[r] * a.scale;
+      }
+#pragma unroll
+      for (int r = 0; r < kSelRows; ++r) acc[r] = 0.f;
     }
   }
   __syncthreads();
@@ -398,7 +545,8 @@ __global__ void compact_kernel(const uint8_t* mask, int32_t* kv_idx, int32_t* kv
 }
 
 template <int D, bool BF16>
-cudaError_t predict_impl(const sparge_params_t& p, const PredictPtrs& x, cudaStream_t s) {
+cudaError_t pool_impl(const sparge_params_t& p, const PredictPtrs& x, cudaStream_t s) {
+  if (p.bq != kPoolBQ || p.bk != kPoolBK) return cudaErrorInvalidValue;
   const int64_t Tm = cdiv(p.N, p.bq), Tn = cdiv(p.N, p.bk);
   PoolArgs pa{};
   pa.q = x.q;
@@ -408,8 +556,9 @@ cudaError_t predict_impl(const sparge_params_t& p, const PredictPtrs& x, cudaStr
   pa.bk = p.bk;
   pa.Tm = int32_t(Tm);
   pa.Tn = int32_t(Tn);
+  const int64_t nK = int64_t(p.B) * p.Hkv * Tn;
   pa.nQblocks = int64_t(p.B) * p.Hq * Tm;
-  pa.nblocks = pa.nQblocks + int64_t(p.B) * p.Hkv * Tn;
+  pa.nblocks = pa.nQblocks + nK;
   pa.q_mean = x.q_mean;
   pa.k_mean = x.k_mean;
   pa.s_q = x.s_q;
@@ -418,24 +567,34 @@ cudaError_t predict_impl(const sparge_params_t& p, const PredictPtrs& x, cudaStr
   pa.dq = x.dq;
   pa.status = x.status;
   cudaError_t e;
-  const int64_t warps_per_cta = kPoolThreads / 32;
-  pool_warp_kernel<D, BF16, 0>
-      <<<unsigned(cdiv(pa.nblocks, warps_per_cta)), kPoolThreads, 0, s>>>(pa);
+  constexpr int SLAB = D == 128 ? 32 : 64;  // 8 KB of bf16/f16 per warp
+  constexpr int64_t warps_per_cta = kPoolThreads / 32;
+  const int64_t w0 = pa.nQblocks * (kPoolBQ / SLAB) + nK * (kPoolBK / SLAB);
+  pool_kernel<D, BF16, 0, SLAB><<<unsigned(cdiv(w0, warps_per_cta)), kPoolThreads, 0, s>>>(pa);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (x.k_codes != nullptr) {
-    kbar_kernel<D><<<unsigned(int64_t(p.B) * p.Hkv), 1024, 0, s>>>(x.k_mean, x.kbar, p.N, p.bk,
-                                                                   int32_t(Tn));
+    const unsigned BHk = unsigned(int64_t(p.B) * p.Hkv);
+    kbar_partial_kernel<D><<<BHk * kKbarSlices, D, 0, s>>>(x.k_mean, x.kbar_part, p.N, p.bk,
+                                                            int32_t(Tn));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    kbar_final_kernel<D><<<BHk, D, 0, s>>>(x.kbar_part, x.kbar, p.N);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     PoolArgs qa = pa;
-    qa.nblocks = int64_t(p.B) * p.Hkv * Tn;
+    qa.nblocks = nK;
     qa.nQblocks = 0;
     qa.kbar = x.kbar;
     qa.k_codes = x.k_codes;
     qa.dk = x.dk;
-    pool_warp_kernel<D, BF16, 1>
-        <<<unsigned(cdiv(qa.nblocks, warps_per_cta)), kPoolThreads, 0, s>>>(qa);
+    const int64_t w1 = nK * (kPoolBK / SLAB);
+    pool_kernel<D, BF16, 1, SLAB><<<unsigned(cdiv(w1, warps_per_cta)), kPoolThreads, 0, s>>>(qa);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  return cudaSuccess;
+}
+
+template <int D>
+cudaError_t select_impl(const sparge_params_t& p, const PredictPtrs& x, cudaStream_t s) {
+  const int64_t Tm = cdiv(p.N, p.bq), Tn = cdiv(p.N, p.bk);
   SelectArgs sa{};
   sa.q_mean = x.q_mean;
   sa.k_mean = x.k_mean;
@@ -456,7 +615,7 @@ cudaError_t predict_impl(const sparge_params_t& p, const PredictPtrs& x, cudaStr
   sa.theta = p.theta;
   sa.scale = p.scale;
   const size_t smem = sizeof(float) * (kSelRows * D + kSelCols * kKPad + kSelRows * Tn);
-  e = cudaFuncSetAttribute(select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            int(smem));
   if (e != cudaSuccess) return e;
   dim3 sgrid{unsigned(cdiv(Tm, kSelRows)), unsigned(p.Hq), unsigned(p.B)};
@@ -466,11 +625,23 @@ cudaError_t predict_impl(const sparge_params_t& p, const PredictPtrs& x, cudaStr
 
 }  // namespace
 
-cudaError_t launch_predict(const sparge_params_t& p, const PredictPtrs& x, cudaStream_t s) {
+cudaError_t launch_predict_pool(const sparge_params_t& p, const PredictPtrs& x, cudaStream_t s) {
   const bool bf16 = p.io_dtype == SPARGE_BF16;
-  if (p.d == 128) return bf16 ? predict_impl<128, true>(p, x, s) : predict_impl<128, false>(p, x, s);
-  if (p.d == 64) return bf16 ? predict_impl<64, true>(p, x, s) : predict_impl<64, false>(p, x, s);
+  if (p.d == 128) return bf16 ? pool_impl<128, true>(p, x, s) : pool_impl<128, false>(p, x, s);
+  if (p.d == 64) return bf16 ? pool_impl<64, true>(p, x, s) : pool_impl<64, false>(p, x, s);
   return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_predict_select(const sparge_params_t& p, const PredictPtrs& x,
+                                  cudaStream_t s) {
+  if (p.d == 128) return select_impl<128>(p, x, s);
+  if (p.d == 64) return select_impl<64>(p, x, s);
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_predict(const sparge_params_t& p, const PredictPtrs& x, cudaStream_t s) {
+  const cudaError_t e = launch_predict_pool(p, x, s);
+  return e != cudaSuccess ? e : launch_predict_select(p, x, s);
 }
 
 cudaError_t launch_mask_compact(const sparge_params_t& p, const uint8_t* mask, int32_t* kv_idx,

@@ -121,22 +121,30 @@ sparge_status_t sparge_inverse_permute(const void* y, void* x, int32_t B, int32_
   return permute_common(y, x, B, H, N, d, dtype, perm, true, stream);
 }
 
-sparge_status_t sparge_predict_mask(const sparge_params_t* p, const void* q, const void* k,
-                                    uint8_t* mask, int32_t* kv_idx, int32_t* kv_cnt, float* s_q,
-                                    float* s_k, void* ws, size_t ws_bytes, cudaStream_t stream) {
+enum : int { kStagePool = 1, kStageSelect = 2 };
+
+// The predictor's entry points share one argument check; `stages` says which
+// half runs (the pooled block statistics travel through the workspace).
+static sparge_status_t predict_common(int stages, const sparge_params_t* p, const void* q,
+                                      const void* k, uint8_t* mask, int32_t* kv_idx,
+                                      int32_t* kv_cnt, float* s_q, float* s_k, void* ws,
+                                      size_t ws_bytes, cudaStream_t stream) {
   sparge_status_t st = check_params(p);
   if (st != SPARGE_OK) return st;
   if (empty_problem(p)) return SPARGE_OK;
-  if (q == nullptr || k == nullptr || mask == nullptr || kv_idx == nullptr || kv_cnt == nullptr ||
-      ws == nullptr)
-    return SPARGE_EINVAL;
-  if (!aligned16(q) || !aligned16(k) || (reinterpret_cast<uintptr_t>(ws) & 255u) ||
-      (reinterpret_cast<uintptr_t>(kv_idx) & 3u) || (reinterpret_cast<uintptr_t>(kv_cnt) & 3u) ||
-      (reinterpret_cast<uintptr_t>(s_q) & 3u) || (reinterpret_cast<uintptr_t>(s_k) & 3u))
-    return SPARGE_EINVAL;
+  if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SPARGE_EINVAL;
+  if (stages & kStagePool) {
+    if (q == nullptr || k == nullptr || !aligned16(q) || !aligned16(k)) return SPARGE_EINVAL;
+  }
+  if (stages & kStageSelect) {
+    if (mask == nullptr || kv_idx == nullptr || kv_cnt == nullptr) return SPARGE_EINVAL;
+    if ((reinterpret_cast<uintptr_t>(kv_idx) & 3u) || (reinterpret_cast<uintptr_t>(kv_cnt) & 3u) ||
+        (reinterpret_cast<uintptr_t>(s_q) & 3u) || (reinterpret_cast<uintptr_t>(s_k) & 3u))
+      return SPARGE_EINVAL;
+  }
   const WsLayout L = ws_layout(*p);
   if (ws_bytes < L.total) return SPARGE_EWORKSPACE;
-  if ((st = select_device(q)) != SPARGE_OK) return st;
+  if ((st = select_device((stages & kStagePool) ? q : ws)) != SPARGE_OK) return st;
   PredictPtrs x{};
   x.q = q;
   x.k = k;
@@ -150,12 +158,18 @@ sparge_status_t sparge_predict_mask(const sparge_params_t* p, const void* q, con
     x.dq = ws_ptr<float>(ws, L.dq);
     x.dk = ws_ptr<float>(ws, L.dk);
     x.kbar = ws_ptr<float>(ws, L.kbar);
+    x.kbar_part = ws_ptr<float>(ws, L.kbar_part);
   }
   x.mask = mask;
   x.kv_idx = kv_idx;
   x.kv_cnt = kv_cnt;
   x.status = ws_ptr<int32_t>(ws, L.status);
-  cudaError_t e = launch_predict(*p, x, stream);
+  if (stages & kStagePool) {
+    const cudaError_t e = launch_predict_pool(*p, x, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+  if (!(stages & kStageSelect)) return SPARGE_OK;
+  const cudaError_t e = launch_predict_select(*p, x, stream);
   if (e != cudaSuccess) return from_cuda(e);
   const int64_t Tm = cdiv(p->N, p->bq), Tn = cdiv(p->N, p->bk);
   if (s_q != nullptr &&
@@ -167,6 +181,26 @@ sparge_status_t sparge_predict_mask(const sparge_params_t* p, const void* q, con
                       stream) != cudaSuccess)
     return SPARGE_ECUDA;
   return SPARGE_OK;
+}
+
+sparge_status_t sparge_predict_mask(const sparge_params_t* p, const void* q, const void* k,
+                                    uint8_t* mask, int32_t* kv_idx, int32_t* kv_cnt, float* s_q,
+                                    float* s_k, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  return predict_common(kStagePool | kStageSelect, p, q, k, mask, kv_idx, kv_cnt, s_q, s_k, ws,
+                        ws_bytes, stream);
+}
+
+sparge_status_t sparge_predict_pool(const sparge_params_t* p, const void* q, const void* k,
+                                    void* ws, size_t ws_bytes, cudaStream_t stream) {
+  return predict_common(kStagePool, p, q, k, nullptr, nullptr, nullptr, nullptr, nullptr, ws,
+                        ws_bytes, stream);
+}
+
+sparge_status_t sparge_predict_select(const sparge_params_t* p, uint8_t* mask, int32_t* kv_idx,
+                                      int32_t* kv_cnt, float* s_q, float* s_k, void* ws,
+                                      size_t ws_bytes, cudaStream_t stream) {
+  return predict_common(kStageSelect, p, nullptr, nullptr, mask, kv_idx, kv_cnt, s_q, s_k, ws,
+                        ws_bytes, stream);
 }
 
 sparge_status_t sparge_mask_compact(const sparge_params_t* p, const uint8_t* mask,

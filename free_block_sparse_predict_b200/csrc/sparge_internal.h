@@ -13,6 +13,8 @@ namespace sparge {
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+constexpr int kKbarSlices = 32;  // key-block slices of the two-level kbar sum
+
 // Offsets (bytes) of every region of the caller's workspace.
 struct WsLayout {
   size_t status;    // int32 status word (kernels OR/CAS error codes in)
@@ -26,6 +28,7 @@ struct WsLayout {
   size_t dq;        // [B, Hq, Tm] f32
   size_t dk;        // [B, Hkv, Tn] f32
   size_t kbar;      // [B, Hkv, d] f32
+  size_t kbar_part; // [B, Hkv, kKbarSlices, d] f32 partial sums of kbar
   size_t total;
   static constexpr size_t npos = ~size_t(0);
 };
@@ -51,8 +54,9 @@ inline WsLayout ws_layout(const sparge_params_t& p) {
     w.dq = take(size_t(p.B) * p.Hq * Tm * 4);
     w.dk = take(size_t(p.B) * p.Hkv * Tn * 4);
     w.kbar = take(size_t(p.B) * p.Hkv * p.d * 4);
+    w.kbar_part = take(size_t(p.B) * p.Hkv * kKbarSlices * p.d * 4);
   } else {
-    w.q_codes = w.k_codes = w.dq = w.dk = w.kbar = WsLayout::npos;
+    w.q_codes = w.k_codes = w.dq = w.dk = w.kbar = w.kbar_part = WsLayout::npos;
   }
   w.total = off;
   return w;
@@ -76,11 +80,17 @@ struct PredictPtrs {
   float* dq;
   float* dk;
   float* kbar;
+  float* kbar_part;
   uint8_t* mask;
   int32_t* kv_idx;
   int32_t* kv_cnt;
   int32_t* status;  // device status word (timeouts of the bounded waits)
 };
+// pooling, self-similarity and INT8 codes (writes the workspace regions) ...
+cudaError_t launch_predict_pool(const sparge_params_t& p, const PredictPtrs& ptrs, cudaStream_t s);
+// ... then S_hat, TopCdf, the fix rule and the skip list from them
+cudaError_t launch_predict_select(const sparge_params_t& p, const PredictPtrs& ptrs,
+                                  cudaStream_t s);
 cudaError_t launch_predict(const sparge_params_t& p, const PredictPtrs& ptrs, cudaStream_t s);
 cudaError_t launch_mask_compact(const sparge_params_t& p, const uint8_t* mask, int32_t* kv_idx,
                                 int32_t* kv_cnt, cudaStream_t s);

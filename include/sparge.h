@@ -127,6 +127,22 @@ sparge_status_t sparge_predict_mask(const sparge_params_t* p, const void* q, con
                                     uint8_t* mask, int32_t* kv_idx, int32_t* kv_cnt, float* s_q,
                                     float* s_k, void* ws, size_t ws_bytes, cudaStream_t stream);
 
+/* The two halves of sparge_predict_mask, for callers that time or schedule
+ * them apart.  sparge_predict_pool is Algorithm 1 steps 2-3 (Eq. 4-6): block
+ * means, CosSim self-similarities and, with qk_int8, the INT8 codes of Q and
+ * K - mean(K) with their scales, all written into ws (the HBM-bound pass over
+ * Q and K).  sparge_predict_select is steps 4-5 (Eq. 7-9): S_hat, softmax,
+ * TopCdf, the fix rule, mask / kv_idx / kv_cnt (and the optional s_q, s_k
+ * copies) computed from what sparge_predict_pool left in the same ws, which
+ * must therefore run first on the same stream (or be ordered before it).
+ * Arguments, layouts and errors as for sparge_predict_mask; pool checks q and
+ * k, select checks the outputs. */
+sparge_status_t sparge_predict_pool(const sparge_params_t* p, const void* q, const void* k,
+                                    void* ws, size_t ws_bytes, cudaStream_t stream);
+sparge_status_t sparge_predict_select(const sparge_params_t* p, uint8_t* mask, int32_t* kv_idx,
+                                      int32_t* kv_cnt, float* s_q, float* s_k, void* ws,
+                                      size_t ws_bytes, cudaStream_t stream);
+
 /* sparge_predict_mask without a workspace, for callers that cannot allocate
  * device memory at call time and have no workspace to pass in (a plugin whose
  * host framework owns every device buffer, a serving loop that must not call

@@ -123,7 +123,8 @@ def ws_regions(p):
     if p.qk_int8:
         for name, nbytes in (("q_codes", p.B * p.Hq * p.N * p.d),
                              ("k_codes", p.B * p.Hkv * p.N * p.d), ("dq", p.B * p.Hq * Tm * 4),
-                             ("dk", p.B * p.Hkv * Tn * 4), ("kbar", p.B * p.Hkv * p.d * 4)):
+                             ("dk", p.B * p.Hkv * Tn * 4), ("kbar", p.B * p.Hkv * p.d * 4),
+                             ("kbar_part", p.B * p.Hkv * 32 * p.d * 4)):
             out[name] = off
             off += al(nbytes)
     return out

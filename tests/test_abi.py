@@ -88,6 +88,14 @@ def test_null_pointers_and_small_workspace(native):
                                  None) == 1
     assert L.sparge_predict_mask(ctypes.byref(p), None, fake, fake, fake, fake, None, None, fake,
                                  1 << 40, None) == 1
+    # the two halves of the predictor check their own arguments
+    assert L.sparge_predict_pool(ctypes.byref(p), None, fake, fake, 1 << 40, None) == 1
+    assert L.sparge_predict_pool(ctypes.byref(p), fake, fake, None, 1 << 40, None) == 1
+    assert L.sparge_predict_pool(ctypes.byref(p), fake, fake, fake, 1024, None) == 5
+    assert L.sparge_predict_select(ctypes.byref(p), None, fake, fake, None, None, fake, 1 << 40,
+                                   None) == 1
+    assert L.sparge_predict_select(ctypes.byref(p), fake, fake, fake, None, None, fake, 1024,
+                                   None) == 5
     assert L.sparge_attn_fwd(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, 1024,
                              None, None) == 5
     misaligned = ctypes.c_void_p(0x10008)

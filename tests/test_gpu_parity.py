@@ -104,6 +104,31 @@ def test_predict_mask_llm_128k_full():
     assert np.array_equal(cnt.cpu().numpy(), M.sum(-1))
 
 
+@pytest.mark.parametrize("name", ["tiny", "llm_128k"])
+def test_predict_pool_then_select_equals_predict_mask(name):
+    # the two halves, called apart on one workspace, give the whole call's
+    # outputs bit for bit (INT8 codes included)
+    over = {"N": 8192 + 100, "Hq": 4, "Hkv": 1} if name == "llm_128k" else {}
+    w, t = workload(name, **over)
+    p = params_for(w)
+    q, k = to_dev(t["q"], w.dtype), to_dev(t["k"], w.dtype)
+    ws, mask, idx, cnt, sq, sk = gpu_predict(p, q, k)
+    ws2 = fb.workspace(p, dev())
+    m2, i2, c2, sq2, sk2 = fb.predict_outputs(p, dev())
+    fb.sparge_predict_pool(p, q, k, ws2)
+    fb.sparge_predict_select(p, m2, i2, c2, sq2, sk2, ws2)
+    torch.cuda.synchronize()
+    assert torch.equal(mask, m2) and torch.equal(cnt, c2)
+    assert torch.equal(sq, sq2) and torch.equal(sk, sk2)
+    for r in range(cnt.numel()):
+        n = int(cnt.view(-1)[r])
+        assert torch.equal(idx.view(-1, idx.shape[-1])[r, :n], i2.view(-1, i2.shape[-1])[r, :n])
+    if w.qk_int8:
+        reg = ws_regions(p)
+        a, b = reg["q_codes"], reg["kbar_part"]
+        assert torch.equal(ws[a:b], ws2[a:b])
+
+
 @pytest.mark.parametrize("tau,theta", [(1.0, 0.5), (0.3, -1.5), (0.5, 1.5), (0.7, 0.0)])
 def test_predict_hyperparameter_limits(tau, theta):
     # tau = 1 keeps every finite block, theta > 1 makes every block a fix
