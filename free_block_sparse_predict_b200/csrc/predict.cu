@@ -124,12 +124,15 @@ __device__ __forceinline__ uint2 codes8(const uint64_t (&x2)[4], float inv) {
 // One warp per SLAB-row slab of a block, held in registers for the whole
 // pass, so every byte of Q and K is read from HBM exactly once per pass.
 // Lane (ro, c) owns the 16-byte chunk c of rows ro, ro + RPW, ...  Arithmetic
-// runs on packed fp32 pairs; the squared row norms of a lane's NR rows are
-// reduced over the CH lanes of each row by a transposing butterfly (each step
-// halves the rows a lane carries), and the inverse norms broadcast back.  The
-// G = block rows / SLAB warps of one block are adjacent in the CTA and combine
-// their partial sums and absmax through shared memory (one named barrier),
-// always in slab order, so the result does not depend on scheduling.
+// runs on packed fp32 pairs in two sweeps over the registers: the first takes
+// the squared row norms, the column sums of x and the exact |x| max; the
+// second, once the block's absmax is known, the column sums of x / |x_row|
+// and the INT8 codes.  The row norms are reduced over the CH lanes of each row
+// by a transposing butterfly (each step halves the rows a lane carries) and
+// the inverse norms broadcast back.  The G = block rows / SLAB warps of one
+// block are adjacent in the CTA and combine their partial sums and absmax
+// through shared memory (named barriers), always in slab order, so the result
+// does not depend on scheduling.
 //   KIND 0  pooling pass over Q blocks then K blocks: mean token, CosSim by
 //           |sum xhat|^2 / n^2, and with q_codes the INT8 codes of Q.
 //   KIND 1  INT8 pass over K blocks: codes of K - kbar and their scales.
@@ -182,9 +185,17 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
 #pragma unroll
   for (int e = 0; e < 8; ++e) sx[e] = su[e] = 0.f;
   float amax = 0.f;
+  float inv_own[R];
+  const int group_base = lane & ~(CH - 1);
+  const int w0 = warp - sub;
   if (KIND == 0) {
-    // ---- squared row norms, one value per row
+    // ---- pass 1: squared row norms (one value per row), column sums of x,
+    // and the exact |x| max on the raw 16-bit halves
     float v[NR];
+    uint64_t sx2[4];
+    uint32_t am2[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sx2[e] = pack2(0.f, 0.f);
 #pragma unroll
     for (int u = 0; u < NR; ++u) {
       const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
@@ -193,11 +204,17 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
       for (int e = 0; e < 4; ++e) {
         const uint64_t x2 = widen2<BF16>(w[e]);
         acc = fma2(x2, x2, acc);
+        sx2[e] = add2(sx2[e], x2);
+        am2[e] = absmax2<BF16>(am2[e], w[e]);
       }
       float s0, s1;
       unpack2(acc, s0, s1);
       v[u] = s0 + s1;
     }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) unpack2(sx2[e], sx[2 * e], sx[2 * e + 1]);
+    amax = absmax2_value<BF16>(absmax2<BF16>(absmax2<BF16>(am2[0], am2[1]),
+                                             absmax2<BF16>(am2[2], am2[3])));
     // ---- butterfly over the CH lanes of a row: at offset o the lanes with
     // bit o set keep the upper half of their rows and send the lower half
 #pragma unroll
@@ -211,36 +228,8 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
       }
     }
     // lane c of a row group now holds rows c * R .. c * R + R - 1
-    float inv_own[R];
 #pragma unroll
     for (int t = 0; t < R; ++t) inv_own[t] = v[t] > 0.f ? rsqrtf(v[t]) : 0.f;
-    const int group_base = lane & ~(CH - 1);
-    // ---- column sums of x and of x / |x_row|, and the exact |x| max
-    uint64_t sx2[4], su2[4];
-    uint32_t am2[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-    for (int e = 0; e < 4; ++e) sx2[e] = su2[e] = pack2(0.f, 0.f);
-#pragma unroll
-    for (int u = 0; u < NR; ++u) {
-      const float inv = __shfl_sync(0xffffffffu, inv_own[u % R], group_base | (u / R));
-      const uint64_t iv2 = pack2(inv, inv);
-      const uint4 rw = opaque(raw[u]);
-      const uint32_t w[4] = {rw.x, rw.y, rw.z, rw.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint64_t x2 = widen2<BF16>(w[e]);
-        sx2[e] = add2(sx2[e], x2);
-        su2[e] = fma2(x2, iv2, su2[e]);
-        am2[e] = absmax2<BF16>(am2[e], w[e]);
-      }
-    }
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      unpack2(sx2[e], sx[2 * e], sx[2 * e + 1]);
-      unpack2(su2[e], su[2 * e], su[2 * e + 1]);
-    }
-    amax = absmax2_value<BF16>(absmax2<BF16>(absmax2<BF16>(am2[0], am2[1]),
-                                             absmax2<BF16>(am2[2], am2[3])));
   } else {
 #pragma unroll
     for (int u = 0; u < NR; ++u) {
@@ -261,71 +250,86 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
 #pragma unroll
     for (int o = CH; o < 32; o <<= 1)
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        sx[e] += __shfl_xor_sync(0xffffffffu, sx[e], o);
-        su[e] += __shfl_xor_sync(0xffffffffu, su[e], o);
-      }
+      for (int e = 0; e < 8; ++e) sx[e] += __shfl_xor_sync(0xffffffffu, sx[e], o);
   }
+  // ---- the block's absmax and column sums over its G slabs (slab order)
   if (G > 1) {
     if (KIND == 0 && ro == 0) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        part[warp][c * 8 + e] = sx[e];
-        part[warp][D + c * 8 + e] = su[e];
-      }
+      for (int e = 0; e < 8; ++e) part[warp][c * 8 + e] = sx[e];
     }
     if (lane == 0) pmax[warp] = amax;
     named_barrier(1 + warp / G, 32 * G);
-    const int w0 = warp - sub;
     if (KIND == 0) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        sx[e] = part[w0][c * 8 + e];
-        su[e] = part[w0][D + c * 8 + e];
-      }
+      for (int e = 0; e < 8; ++e) sx[e] = part[w0][c * 8 + e];
       for (int g = 1; g < G; ++g)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          sx[e] += part[w0 + g][c * 8 + e];
-          su[e] += part[w0 + g][D + c * 8 + e];
-        }
+        for (int e = 0; e < 8; ++e) sx[e] += part[w0 + g][c * 8 + e];
     }
     amax = pmax[w0];
     for (int g = 1; g < G; ++g) amax = fmaxf(amax, pmax[w0 + g]);
   }
-  if (KIND == 0 && sub == 0) {
-    float uu = 0.f;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) uu = fmaf(su[e], su[e], uu);
-#pragma unroll
-    for (int o = CH / 2; o > 0; o >>= 1) uu += __shfl_xor_sync(0xffffffffu, uu, o);
-    float* mean = isQ ? a.q_mean : a.k_mean;
-    if (lane < CH) {
-      const float n = float(rows);
-      float4* dst = reinterpret_cast<float4*>(mean + (bh * T + blk) * D + c * 8);
-      dst[0] = make_float4(sx[0] / n, sx[1] / n, sx[2] / n, sx[3] / n);
-      dst[1] = make_float4(sx[4] / n, sx[5] / n, sx[6] / n, sx[7] / n);
-    }
-    if (lane == 0) (isQ ? a.s_q : a.s_k)[bh * T + blk] = uu / (float(rows) * float(rows));
-  }
   const bool quantise = KIND == 1 || (isQ && a.q_codes != nullptr);
-  if (!quantise) return;
   const float inv = amax > 0.f ? 127.0f / amax : 0.f;
-  if (sub == 0 && lane == 0) (KIND == 1 ? a.dk : a.dq)[bh * T + blk] = amax / 127.0f;
-  int8_t* codes = (KIND == 1 ? a.k_codes : a.q_codes) + row0 * D + c * 8;
+  if (quantise && sub == 0 && lane == 0) (KIND == 1 ? a.dk : a.dq)[bh * T + blk] = amax / 127.0f;
+  int8_t* codes = quantise ? (KIND == 1 ? a.k_codes : a.q_codes) + row0 * D + c * 8 : nullptr;
+  // ---- pass 2: column sums of x / |x_row| (and the codes, once absmax is known)
+  uint64_t su2[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) su2[e] = pack2(0.f, 0.f);
 #pragma unroll
   for (int u = 0; u < NR; ++u) {
     const int r = ro + u * RPW;
-    if (r < srows) {
-      const uint4 rw = opaque(raw[u]);
-      const uint32_t w[4] = {rw.x, rw.y, rw.z, rw.w};
-      uint64_t x2[4];
+    const uint4 rw = opaque(raw[u]);
+    const uint32_t w[4] = {rw.x, rw.y, rw.z, rw.w};
+    uint64_t x2[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        x2[e] = widen2<BF16>(w[e]);
-        if (KIND == 1) x2[e] = add2(x2[e], nkb2[e]);
+    for (int e = 0; e < 4; ++e) x2[e] = widen2<BF16>(w[e]);
+    if (KIND == 0) {
+      const float iv = __shfl_sync(0xffffffffu, inv_own[u % R], group_base | (u / R));
+      const uint64_t iv2 = pack2(iv, iv);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) su2[e] = fma2(x2[e], iv2, su2[e]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) x2[e] = add2(x2[e], nkb2[e]);
+    }
+    if (quantise && r < srows) *reinterpret_cast<uint2*>(codes + int64_t(r) * D) = codes8(x2, inv);
+  }
+  if constexpr (KIND == 0) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) unpack2(su2[e], su[2 * e], su[2 * e + 1]);
+#pragma unroll
+    for (int o = CH; o < 32; o <<= 1)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) su[e] += __shfl_xor_sync(0xffffffffu, su[e], o);
+    if (G > 1) {
+      if (ro == 0) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) part[warp][D + c * 8 + e] = su[e];
       }
-      *reinterpret_cast<uint2*>(codes + int64_t(r) * D) = codes8(x2, inv);
+      named_barrier(1 + warp / G, 32 * G);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) su[e] = part[w0][D + c * 8 + e];
+      for (int g = 1; g < G; ++g)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) su[e] += part[w0 + g][D + c * 8 + e];
+    }
+    if (sub == 0) {
+      float uu = 0.f;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) uu = fmaf(su[e], su[e], uu);
+#pragma unroll
+      for (int o = CH / 2; o > 0; o >>= 1) uu += __shfl_xor_sync(0xffffffffu, uu, o);
+      float* mean = isQ ? a.q_mean : a.k_mean;
+      if (lane < CH) {
+        const float n = float(rows);
+        float4* dst = reinterpret_cast<float4*>(mean + (bh * T + blk) * D + c * 8);
+        dst[0] = make_float4(sx[0] / n, sx[1] / n, sx[2] / n, sx[3] / n);
+        dst[1] = make_float4(sx[4] / n, sx[5] / n, sx[6] / n, sx[7] / n);
+      }
+      if (lane == 0) (isQ ? a.s_q : a.s_k)[bh * T + blk] = uu / (float(rows) * float(rows));
     }
   }
 }
