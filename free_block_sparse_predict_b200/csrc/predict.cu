@@ -10,8 +10,8 @@
 //   pool_kernel<.., 1>  per-block INT8 of K - kbar (second pass over K).
 //   select_kernel   per query block: S_hat = scale q_i k^T with -inf columns
 //                   (Eq. 7), row softmax, TopCdf(tau) (Eq. 8) by an exact
-//                   value-threshold bisection, the fix-block rule (Eq. 9), and
-//                   the ascending per-tile skip list.
+//                   radix select of the threshold value, the fix-block rule
+//                   (Eq. 9), and the ascending per-tile skip list.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -379,16 +379,15 @@ struct SelectArgs {
   float tau, theta, scale;
 };
 
+// e * 2^40 as an integer (e in [0, 1]); exact for e >= 2^-16
+__device__ __forceinline__ unsigned long long fixed40(float e) {
+  return __float2ull_rz(e * 1099511627776.0f);
+}
+
 __device__ __forceinline__ int visible_cols(int i, int N, int bq, int bk, int Tn, int causal) {
   if (!causal) return Tn;
   const int last_row = min(N, (i + 1) * bq) - 1;
   return min(Tn, last_row / bk + 1);
-}
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
 }
 
 template <int D>
@@ -483,36 +482,78 @@ __global__ void __launch_bounds__(256) select_kernel(SelectArgs a) {
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  // unnormalised softmax weights; -1 marks a -inf entry
-  float tot = 0.f;
+  // unnormalised softmax weights; -1 marks a -inf entry.  Each weight's mass
+  // is also taken as the integer e * 2^40 (exact for e >= 2^-16, below that
+  // truncated by < 2^-40), so that every partial sum below is exact and does
+  // not depend on the order of summation.
+  unsigned long long tot = 0ull;
   for (int j = lane; j < nvis; j += 32) {
     const float v = row[j];
     const float e = (v == -INFINITY) ? -1.f : expf(v - mx);
     row[j] = e;
-    tot += fmaxf(e, 0.f);
+    if (e >= 0.f) tot += fixed40(e);
   }
-  tot = warp_sum(tot);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
   __syncwarp();
   float t_star = 0.f;  // keep e >= t_star (t_star = 0 keeps every finite entry)
   if (a.tau < 1.0f) {
-    // largest t with sum_{e >= t} e >= tau * total: an exact value of the row
-    const float target = a.tau * tot;
-    uint32_t lo = 0u, hi = 0x3F800001u;  // f(lo) >= target, f(hi) = 0 < target
-    while (hi - lo > 1u) {
-      const uint32_t mid = lo + ((hi - lo) >> 1);
-      const float t = __uint_as_float(mid);
-      float f = 0.f;
+    // t* = the largest row value t with sum_{e >= t} e >= tau * total, by a
+    // radix select on the bit patterns of e (ordered like the values for
+    // e >= 0), most significant byte first: each pass histograms the masses
+    // of the entries that share the prefix found so far and picks the digit
+    // where the running sum from the top reaches the target.
+    const unsigned long long target =
+        static_cast<unsigned long long>(ceil(double(a.tau) * double(tot)));
+    unsigned long long* hist = reinterpret_cast<unsigned long long*>(ks) + w * 256;
+    uint32_t prefix = 0u;
+    unsigned long long above = 0ull;  // mass of the entries above the prefix's range
+#pragma unroll 1
+    for (int shift = 24; shift >= 0; shift -= 8) {
+      const uint32_t pmask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
+#pragma unroll
+      for (int b = 0; b < 8; ++b) hist[lane * 8 + b] = 0ull;
+      __syncwarp();
       for (int j = lane; j < nvis; j += 32) {
         const float e = row[j];
-        f += (e >= t) ? e : 0.f;
+        const uint32_t key = __float_as_uint(e);
+        if (e >= 0.f && (key & pmask) == prefix)
+          atomicAdd(hist + ((key >> shift) & 255u), fixed40(e));
       }
-      f = warp_sum(f);
-      if (f >= target)
-        lo = mid;
-      else
-        hi = mid;
+      __syncwarp();
+      // lane L holds digits 8L .. 8L+7; suffix sums over lanes from the top
+      unsigned long long h[8], mine = 0ull;
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        h[b] = hist[lane * 8 + b];
+        mine += h[b];
+      }
+      unsigned long long incl = mine;  // mass of lanes >= this lane
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long up = __shfl_down_sync(0xffffffffu, incl, o);
+        if (lane + o < 32) incl += up;
+      }
+      const unsigned ok = __ballot_sync(0xffffffffu, above + incl >= target);
+      const int L = ok ? 31 - __clz(ok) : 0;  // the highest lane that reaches it
+      uint32_t digit = 0u;
+      unsigned long long run = above + incl - mine;  // mass above lane L's digits
+      if (lane == L) {
+#pragma unroll
+        for (int b = 7; b >= 0; --b) {
+          if (run + h[b] >= target) {
+            digit = uint32_t(8 * L + b);
+            break;
+          }
+          run += h[b];
+        }
+      }
+      digit = __shfl_sync(0xffffffffu, digit, L);
+      above = __shfl_sync(0xffffffffu, run, L);
+      prefix |= digit << shift;
+      __syncwarp();
     }
-    t_star = __uint_as_float(lo);
+    t_star = tot == 0ull ? INFINITY : __uint_as_float(prefix);
   }
   const int64_t out = (bh * a.Tm + i) * a.Tn;
   int cnt = 0;
