@@ -171,14 +171,19 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const __grid_constant
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- tile of this CTA: heavy (late) query blocks first, heads of one KV
-  // group adjacent so they share K/V through L2
-  const int64_t BH = int64_t(P.B) * P.Hq;
-  const int i = P.Tm - 1 - int(blockIdx.x / BH);
-  const int64_t bh = blockIdx.x % BH;
-  const int b = int(bh / P.Hq), h = int(bh % P.Hq);
-  const int hk = h / (P.Hq / P.Hkv);
-  const int64_t bhk = int64_t(b) * P.Hkv + hk;
+  // ---- tile of this CTA.  Tiles are ordered by (batch, KV head) first, so
+  // the CTAs resident at any time read the K/V of one KV head, which then
+  // stays in L2 (50 MB at N = 128K, d = 128) instead of all heads' streaming
+  // through it; within a KV head, heavy (late) query blocks first, and the
+  // query heads of the group adjacent.
+  const int G = P.Hq / P.Hkv;
+  const int64_t per_kv = int64_t(P.Tm) * G;
+  const int64_t bhk = blockIdx.x / per_kv;
+  const int64_t rem = blockIdx.x % per_kv;
+  const int i = P.Tm - 1 - int(rem / G);
+  const int b = int(bhk / P.Hkv), hk = int(bhk % P.Hkv);
+  const int h = hk * G + int(rem % G);
+  const int64_t bh = int64_t(b) * P.Hq + h;
   const int64_t tile = bh * P.Tm + i;
   const int32_t* kv_list = P.kv_idx + tile * P.Tn;
   int n = P.kv_cnt[tile];
