@@ -22,7 +22,8 @@
  *              synchronises except sparge_device_status.
  *   Errors     Arguments are validated on the host before any launch:
  *              SPARGE_EINVAL (bad pointer, size or hyper-parameter),
- *              SPARGE_EUNSUPPORTED (valid but not implemented, e.g. d = 96),
+ *              SPARGE_EUNSUPPORTED (valid but not implemented, e.g. d = 96,
+ *              b_q != 128, b_k != 64, or more than 5952 key blocks: N > 380,928),
  *              SPARGE_EWORKSPACE (workspace too small), SPARGE_ECUDA (a CUDA
  *              runtime call or launch failed).  Nothing is launched when a call
  *              returns an error.  Kernels never trap: a device-side wait that

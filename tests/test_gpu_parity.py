@@ -188,6 +188,33 @@ def test_attention_fp32_output_matches_oracle(name, over, tph, heads):
         assert abs(int(st[4]) - ost["skipped_slices"]) <= ost["near_lambda"]
 
 
+@pytest.mark.parametrize("name", ["llm_32k", "llm_128k"])
+def test_batched_gqa_with_ragged_tail(name):
+    # B = 2, GQA 2:1 and a ragged last block: the tile, batch and KV-head
+    # indexing of every kernel (pooling, select, attention's KV-head-major tile
+    # order) across batches, in 16-bit and INT8 modes, against the oracle
+    over = dict(N=2048 + 40, B=2, Hq=4, Hkv=2)
+    w, t = workload(name, **over)
+    Q, K, _ = oracle_inputs(w, t)
+    p = params_for(w)
+    ws, mask, idx, cnt, sq, sk = gpu_predict(p, to_dev(t["q"], w.dtype), to_dev(t["k"], w.dtype))
+    pr = orc.predict_mask(Q, K, w.bq, w.bk, w.tau, w.theta, w.causal, w.scale)
+    M = mask.cpu().numpy().astype(bool)
+    assert not ((M != pr["M"]) & ~pr["amb"]).any()
+    assert np.abs(sq.cpu().numpy() - pr["s_q"]).max() < 1e-5
+    w, o, O, ost, st, rows = _attention_case(name, over)
+    if w.qk_int8:
+        l1 = np.abs(o - O).sum() / np.abs(O).sum()
+        cos = (o * O).sum() / np.linalg.norm(o) / np.linalg.norm(O)
+        assert l1 <= INT8_REL_L1 and cos >= INT8_COS, (l1, cos)
+    else:
+        mx, l1 = compare_rows(o, O, rows, exclude=ost["near_rows"])
+        assert mx <= MAX_ABS and l1 <= MEAN_REL_L1, (mx, l1, ost["near_lambda"])
+        assert st[1] == ost["qk_blocks"]
+    # the two batches differ, and so must their outputs
+    assert not np.allclose(o[0], o[1])
+
+
 def test_attention_16bit_output_is_rounded_fp32_result():
     # the 16-bit output mode differs from the float32 mode only in the
     # epilogue store: it must be exactly the round-to-nearest-even of the
