@@ -1,0 +1,69 @@
+"""bench.py's accounting and its reference arm, on the CPU.
+
+The pooling stage's algorithmic bytes are pinned to a hand count for the 128K
+INT8 workload (B1 Hq32 Hkv8 N131072 d128 bf16), term by term, so a dropped or
+doubled term in the roofline's numerator fails here; the reference arm (the
+float64 oracle on a bounded sample) must print one JSON line with the fields
+the driver reads.
+"""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from synth import get_workload  # noqa: E402
+
+
+def test_pool_bytes_hand_count_128k_int8():
+    w = get_workload("llm_128k")
+    q = 32 * 131072 * 128 * 2            # read Q (bf16)
+    k = 8 * 131072 * 128 * 2             # read K
+    means = (32 * 1024 + 8 * 2048) * (128 + 1) * 4   # block means and self-similarities
+    q_codes = 32 * 131072 * 128 + 32 * 1024 * 4      # Q codes and their scales
+    kbar = 8 * 2048 * 128 * 4            # k-bar from the K block means
+    k_again = 8 * 131072 * 128 * 2       # second read of K
+    k_codes = 8 * 131072 * 128 + 8 * 2048 * 4        # K codes and their scales
+    assert bench.pool_bytes(w) == q + k + means + q_codes + kbar + k_again + k_codes
+    assert bench.pool_bytes(w) == 2_315_649_024
+
+
+def test_pool_bytes_without_int8_is_one_read_plus_means():
+    w = get_workload("llm_32k")
+    assert bench.pool_bytes(w) == (32 + 8) * 32768 * 128 * 2 + (32 * 256 + 8 * 512) * 129 * 4
+
+
+def test_dense_equivalent_ops_halved_when_causal():
+    w = get_workload("llm_128k")
+    assert bench.dense_equiv_ops(w) == 4.0 * 131072 ** 2 * 128 * 32 / 2
+    t = get_workload("tiny")
+    assert bench.dense_equiv_ops(t) == 4.0 * 1024 ** 2 * 64 * 1
+
+
+def test_visible_blocks_causal_count():
+    # causal: query block i (128 rows) sees key blocks 0 .. 2i+1 (64 rows each)
+    w = get_workload("llm_32k").replace(N=1024, Hq=1, Hkv=1)
+    assert bench._visible_blocks(w) == sum(2 * i + 2 for i in range(8))
+
+
+def test_fp32_peak_from_unit_counts():
+    assert bench.fp32_peak_tflops({"sm_max_mhz": 1965.0}) == pytest.approx(74.45, rel=1e-3)
+
+
+def test_reference_arm_prints_one_json_line():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--workload", "tiny", "--steps", "1", "--warmup", "0", "--ref-tiles", "2"],
+                       capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.strip().startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "TOPS" and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
+    assert d["higher_is_better"] is True and d["n_gpus"] == 1
