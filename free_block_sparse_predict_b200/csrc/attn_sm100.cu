@@ -378,7 +378,10 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const __grid_constant
         uint32_t (&r1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&raw[32]);
         tmem_ld32(lane_addr + uint32_t(sb * kBK), r0);
         tmem_ld32(lane_addr + uint32_t(sb * kBK + 32), r1);
-        tmem_wait_ld();
+        // the fenced waits tie r0 / r1 to the wait, so no use of them can be
+        // scheduled before the loads have landed
+        tmem_wait_ld_fence(r0);
+        tmem_wait_ld_fence(r1);
       }
       // INT8 scores become floats first, without the conversion unit (it
       // shares the MUFU pipe with ex2): the bits of 1.5 * 2^23 + x are that
@@ -415,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const __grid_constant
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
           tmem_ld32(lane_addr + uint32_t(C::O_COL + cc * 32), o);
-          tmem_wait_ld();
+          tmem_wait_ld_fence(o);
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
           tmem_st32(lane_addr + uint32_t(C::O_COL + cc * 32), o);
@@ -486,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const __grid_constant
         uint32_t o[32] = {};
         if (n > 0) {
           tmem_ld32(lane_addr + uint32_t(C::O_COL + cc * 32), o);
-          tmem_wait_ld();
+          tmem_wait_ld_fence(o);
         }
         float v[32];
 #pragma unroll
