@@ -302,6 +302,26 @@ def test_int8_attention_full_128k_sampled_tiles():
 # edge cases
 # ----------------------------------------------------------------------------
 
+def test_maximum_length_mask_and_sampled_tiles():
+    # the largest N the library accepts (5952 key blocks of 64, the select
+    # kernel's shared-memory bound), causal, one head: the whole mask against
+    # the oracle, attention on sampled tiles including the last (5952 blocks)
+    N = 5952 * 64
+    w, t = workload("llm_32k", N=N, Hq=1, Hkv=1)
+    Q, K, _ = oracle_inputs(w, t)
+    p = params_for(w)
+    ws, mask, idx, cnt, sq, sk = gpu_predict(p, to_dev(t["q"], w.dtype), to_dev(t["k"], w.dtype))
+    pr = orc.predict_mask(Q, K, w.bq, w.bk, w.tau, w.theta, w.causal, w.scale)
+    M = mask.cpu().numpy().astype(bool)
+    assert not ((M != pr["M"]) & ~pr["amb"]).any()
+    assert int(cnt.view(-1)[-1]) == M[0, 0, -1].sum() == 5952
+    w, o, O, ost, st, rows = _attention_case("llm_32k", {"N": N, "Hq": 1, "Hkv": 1}, 2, [0])
+    mx, l1 = compare_rows(o, O, rows, exclude=ost["near_rows"])
+    assert mx <= MAX_ABS and l1 <= MEAN_REL_L1, (mx, l1, ost["near_lambda"])
+    # one more key block is refused before anything runs
+    assert fb.sparge_workspace_bytes(params_for(w.replace(N=N + 1))) == 0
+
+
 @pytest.mark.parametrize("N,causal", [(1, False), (1, True), (65, True), (129, False),
                                       (200, True), (1000, False)])
 def test_ragged_and_tiny_lengths(N, causal):
