@@ -363,8 +363,9 @@ __global__ void __launch_bounds__(D) kbar_final_kernel(const float* part, float*
 }
 
 // ------------------------------------------------------------------ select
-constexpr int kSelRows = 8;   // query blocks per CTA (one warp each)
-constexpr int kSelCols = 256; // key blocks scored per pass (one thread each)
+constexpr int kSelRows = 8;                 // query blocks per CTA (one warp each)
+constexpr int kSelThreads = kSelRows * 32;
+constexpr int kSelCols = kSelThreads;       // key blocks scored per pass (one thread each)
 constexpr int kKPad = 36;     // padded row of a staged 32-float k chunk
 
 struct SelectArgs {
@@ -391,7 +392,7 @@ __device__ __forceinline__ int visible_cols(int i, int N, int bq, int bk, int Tn
 }
 
 template <int D>
-__global__ void __launch_bounds__(256) select_kernel(SelectArgs a) {
+__global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
   extern __shared__ __align__(16) float smem[];
   float* qs = smem;                        // [kSelRows][D]
   float* ks = qs + kSelRows * D;           // [kSelCols][kKPad]
@@ -405,7 +406,7 @@ __global__ void __launch_bounds__(256) select_kernel(SelectArgs a) {
   const int i_last = min(a.Tm, i0 + kSelRows) - 1;
   const int jcount = visible_cols(i_last, a.N, a.bq, a.bk, a.Tn, a.causal);
 
-  for (int idx = tid; idx < kSelRows * D; idx += 256) {
+  for (int idx = tid; idx < kSelRows * D; idx += kSelThreads) {
     const int r = idx / D, e = idx % D;
     qs[idx] = (i0 + r < a.Tm) ? a.q_mean[(bh * a.Tm + i0 + r) * D + e] : 0.f;
   }
@@ -416,12 +417,12 @@ __global__ void __launch_bounds__(256) select_kernel(SelectArgs a) {
   // L2 latency of the loads overlaps the arithmetic.
   const int njt = (jcount + kSelCols - 1) / kSelCols;
   const int nchunks = njt * (D / 32);
-  float4 pre[kSelCols * 8 / 256];
+  float4 pre[kSelCols * 8 / kSelThreads];
   auto fetch = [&](int chunk) {
     const int jt = chunk / (D / 32), ec = (chunk % (D / 32)) * 32;
 #pragma unroll
-    for (int u = 0; u < kSelCols * 8 / 256; ++u) {
-      const int idx = tid + u * 256;
+    for (int u = 0; u < kSelCols * 8 / kSelThreads; ++u) {
+      const int idx = tid + u * kSelThreads;
       const int jl = idx >> 3, f4 = idx & 7, j = jt * kSelCols + jl;
       pre[u] = j < jcount
                    ? *reinterpret_cast<const float4*>(a.k_mean + (kbh * a.Tn + j) * D + ec + f4 * 4)
@@ -436,8 +437,8 @@ __global__ void __launch_bounds__(256) select_kernel(SelectArgs a) {
     const int jt = chunk / (D / 32), ec = (chunk % (D / 32)) * 32;
     __syncthreads();  // the previous chunk is no longer read
 #pragma unroll
-    for (int u = 0; u < kSelCols * 8 / 256; ++u) {
-      const int idx = tid + u * 256;
+    for (int u = 0; u < kSelCols * 8 / kSelThreads; ++u) {
+      const int idx = tid + u * kSelThreads;
       *reinterpret_cast<float4*>(ks + (idx >> 3) * kKPad + (idx & 7) * 4) = pre[u];
     }
     __syncthreads();
@@ -664,7 +665,7 @@ cudaError_t select_impl(const sparge_params_t& p, const PredictPtrs& x, cudaStre
                            int(smem));
   if (e != cudaSuccess) return e;
   dim3 sgrid{unsigned(cdiv(Tm, kSelRows)), unsigned(p.Hq), unsigned(p.B)};
-  select_kernel<D><<<sgrid, 256, smem, s>>>(sa);
+  select_kernel<D><<<sgrid, kSelThreads, smem, s>>>(sa);
   return cudaGetLastError();
 }
 
