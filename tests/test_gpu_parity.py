@@ -281,6 +281,28 @@ def test_int8_codes_and_scales_match_oracle():
     assert dk.max() <= 1 and dk.mean() < 1e-3                  # kbar summation order only
 
 
+def test_int8_with_fp16_io_and_ragged_tail():
+    # INT8 Q K^T with fp16 inputs (no V conversion) and a ragged tail: Q codes
+    # and scales bit-exact, the mask against the oracle, the output within the
+    # INT8 bar
+    over = {"N": 2048 + 96, "Hq": 4, "Hkv": 2, "dtype": "f16"}
+    w, t = workload("llm_128k", **over)
+    Q, K, _ = oracle_inputs(w, t)
+    p = params_for(w)
+    ws, mask, idx, cnt, sq, sk = gpu_predict(p, to_dev(t["q"], w.dtype), to_dev(t["k"], w.dtype))
+    reg = ws_regions(p)
+    raw = ws.cpu().numpy()
+    qc = raw[reg["q_codes"]:reg["q_codes"] + Q.size].view(np.int8).reshape(Q.shape)
+    qt = orc.quantize_qk(Q.astype(np.float32), K.astype(np.float32), 128, 64)
+    assert np.array_equal(qc, qt["q_codes"])
+    pr = orc.predict_mask(Q, K, w.bq, w.bk, w.tau, w.theta, w.causal, w.scale)
+    assert not ((mask.cpu().numpy().astype(bool) != pr["M"]) & ~pr["amb"]).any()
+    w, o, O, ost, st, rows = _attention_case("llm_128k", over)
+    l1 = np.abs(o - O).sum() / np.abs(O).sum()
+    cos = (o * O).sum() / np.linalg.norm(o) / np.linalg.norm(O)
+    assert l1 <= INT8_REL_L1 and cos >= INT8_COS, (l1, cos)
+
+
 def test_int8_attention_small_matches_exact_scores():
     w, t = workload("llm_128k", N=4096, Hq=8, Hkv=2)
     w_, o, O, ost, st, rows = _attention_case("llm_128k", {"N": 4096, "Hq": 8, "Hkv": 2})
