@@ -80,15 +80,18 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
-def profiled_traffic():
+def profiled_traffic(workload: str, seq_len: int, path: str = PROFILE_SUMMARY):
     """dram bytes per attention launch from the committed ncu summary, if it
-    was taken on the current kernel source."""
-    if not os.path.exists(PROFILE_SUMMARY):
+    was taken on the current kernel source and on this workload and length."""
+    if not os.path.exists(path):
         return None
-    text = open(PROFILE_SUMMARY).read()
+    text = open(path).read()
     m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
     h = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
-    if not m or not h:
+    wl = re.search(r"dram_bytes_workload:\s*(\S+)\s+N=(\d+)", text)
+    if not m or not h or not wl:
+        return None
+    if wl.group(1) != workload or int(wl.group(2)) != int(seq_len):
         return None
     cur = hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()
     return float(m.group(1)) if h.group(1) == cur else None
@@ -349,7 +352,7 @@ def run_native(args, rank, world, local_rank):
     peaks, peak_src = load_peaks()
     peak = float(peaks["bf16_tflops_sustained"])
     peak_burst = float(peaks["bf16_tflops"])
-    traffic = profiled_traffic()
+    traffic = profiled_traffic(w.name, w.N)
     pbytes = pool_bytes(w)
     hbm_peak = float(peaks["hbm_gbs"])
     sel_flops = 2.0 * w.d * _visible_pairs(w)

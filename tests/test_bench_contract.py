@@ -67,3 +67,18 @@ def test_reference_arm_prints_one_json_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
     assert d["higher_is_better"] is True and d["n_gpus"] == 1
+
+
+def test_profiled_traffic_only_for_the_profiled_workload(tmp_path):
+    import hashlib
+    sha = hashlib.sha256(open(bench.ATTN_SRC, "rb").read()).hexdigest()
+    p = tmp_path / "summary.md"
+    p.write_text(f"kernel_source_sha256: {sha}\ndram_bytes_per_launch: 2.25e9\n"
+                 "dram_bytes_workload: llm_128k N=131072\n")
+    assert bench.profiled_traffic("llm_128k", 131072, str(p)) == 2.25e9
+    # another workload, another length, another kernel source: no figure
+    assert bench.profiled_traffic("image_dit", 4608, str(p)) is None
+    assert bench.profiled_traffic("llm_128k", 32768, str(p)) is None
+    p.write_text("kernel_source_sha256: 00\ndram_bytes_per_launch: 2.25e9\n"
+                 "dram_bytes_workload: llm_128k N=131072\n")
+    assert bench.profiled_traffic("llm_128k", 131072, str(p)) is None
