@@ -427,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const __grid_constant
       }
       if (grow) m_sc = m_new;
       // P~ = 2^(x * sc - m_sc): one packed FMA per pair, then ex2 on the MUFU
-      // for three columns in four and the FMA-pipe polynomial for the fourth
+      // (with kExp2OnFma, the FMA-pipe polynomial for one pair in four)
       const float nb = (m_sc == -INFINITY) ? 0.f : -m_sc;
       const uint64_t sc2 = pack2(sc, sc), nb2 = pack2(nb, nb);
       float pv[64];
