@@ -260,10 +260,13 @@ def run_native(args, rank, world, local_rank):
         sampler.start()
         time.sleep(0.3)
     # inputs that fit in L2 would stay there from one step to the next: then a
-    # 256 MB buffer is rewritten between steps and only the steps are timed
-    flush = None
+    # 256 MB buffer is rewritten between steps and only the steps are timed.
+    # A second 256 MB buffer is read after it, so that the flush's own dirty
+    # lines are written back before the step starts instead of inside it.
+    flush = flush_rd = None
     if _bytes(t) <= L2_BYTES:
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+        flush_rd = torch.ones(256 * 1024 * 1024 // 4, dtype=torch.int32, device=dev)
     e0, e1 = ev(), ev()
     per = [(ev(), ev(), ev(), ev()) for _ in range(args.steps)]
     span = [(ev(), ev()) for _ in range(args.steps)]
@@ -271,6 +274,7 @@ def run_native(args, rank, world, local_rank):
     for s in range(args.steps):
         if flush is not None:
             flush.fill_(s & 255)
+            flush_rd.max()
         span[s][0].record(stream)
         step(q, k, v, o, per[s])
         span[s][1].record(stream)
@@ -283,6 +287,11 @@ def run_native(args, rank, world, local_rank):
     pool_ms = float(np.mean([a.elapsed_time(b) for (a, b, _, _) in per]))
     sel_ms = float(np.mean([a.elapsed_time(b) for (_, a, b, _) in per]))
     attn_ms = float(np.mean([a.elapsed_time(b) for (_, _, a, b) in per]))
+    step_median_ms = float(np.median([a.elapsed_time(b) for a, b in span]))
+    # grid workloads: Hilbert table + permutes of Q, K, V before the predictor,
+    # inverse permute of O after the attention
+    perm_ms = float(np.mean([sp[0].elapsed_time(pe[0]) for sp, pe in zip(span, per)]))
+    inv_ms = float(np.mean([pe[3].elapsed_time(sp[1]) for sp, pe in zip(span, per)]))
     pred_ms = pool_ms + sel_ms
     ms_total = max_over_ranks(ms_total, world, dev)
     ms_step = ms_total / args.steps
@@ -375,10 +384,13 @@ def run_native(args, rank, world, local_rank):
                    "global_batch": w.B * world, "seq_len": w.N,
                    "parallelism": f"replicas x{world}",
                    "l2": "inputs larger than L2 (no flush)" if _bytes(t) > L2_BYTES
-                   else "inputs fit in L2: 256 MB rewritten between steps, steps timed alone"},
+                   else "inputs fit in L2: 256 MB rewritten, then 256 MB read, between "
+                        "steps; steps timed alone"},
         "latency_ms": {"predict": round(pred_ms, 4), "predict_pool": round(pool_ms, 4),
                        "predict_select": round(sel_ms, 4), "attention": round(attn_ms, 4),
-                       "step": round(ms_step, 4)},
+                       "step": round(ms_step, 4), "step_median": round(step_median_ms, 4),
+                       **({"permute": round(perm_ms, 4), "inverse_permute": round(inv_ms, 4)}
+                          if w.grid else {})},
         "predict_roofline": {
             "pool": {"bound": "hbm", "achieved": round(pbytes / (pool_ms * 1e-3) / 1e9, 1),
                      "peak": hbm_peak, "unit": "GB/s",
@@ -386,6 +398,21 @@ def run_native(args, rank, world, local_rank):
                      "bytes_per_launch": pbytes,
                      "kernel": "pool_kernel (+ k-bar and the K-code pass with INT8), "
                                "algorithmic bytes / stage time"},
+            **({"permute": {"bound": "hbm", "unit": "GB/s", "peak": hbm_peak,
+                            "bytes_per_launch": 2 * _bytes(t),
+                            "achieved": round(2 * _bytes(t) / (perm_ms * 1e-3) / 1e9, 1),
+                            "frac": round(2 * _bytes(t) / (perm_ms * 1e-3) / 1e9 / hbm_peak, 4),
+                            "kernel": "Hilbert table + gather of Q, K, V: each read once and "
+                                      "written once / stage time"},
+                "inverse_permute": {"bound": "hbm", "unit": "GB/s", "peak": hbm_peak,
+                                    "bytes_per_launch": 2 * o.numel() * o.element_size(),
+                                    "achieved": round(2 * o.numel() * o.element_size()
+                                                      / (inv_ms * 1e-3) / 1e9, 1),
+                                    "frac": round(2 * o.numel() * o.element_size()
+                                                  / (inv_ms * 1e-3) / 1e9 / hbm_peak, 4),
+                                    "kernel": "scatter of O back to token order: read once, "
+                                              "written once / stage time"}}
+               if w.grid else {}),
             "select": {"bound": "fp32", "achieved": round(sel_flops / (sel_ms * 1e-3) / 1e12, 2),
                        "peak": round(fp32_peak, 1), "unit": "TFLOP/s",
                        "frac": round(sel_flops / (sel_ms * 1e-3) / 1e12 / fp32_peak, 4),

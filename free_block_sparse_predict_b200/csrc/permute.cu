@@ -132,22 +132,47 @@ __global__ void hilbert_scatter_kernel(HilbertGrid g, const int32_t* counts, int
 }
 
 // Whole-row gather (y[p] = x[perm[p]]) or scatter (y[perm[p]] = x[p]) inside
-// each (batch, head) slab; blockIdx.y is the slab.  Rows are moved as
-// 16-byte vectors; table entries outside [0, N) are skipped.
-__global__ void permute_kernel(const uint4* __restrict__ x, uint4* __restrict__ y, int32_t N,
-                               int32_t vpr, const int32_t* __restrict__ perm, int inverse) {
+// each (batch, head) slab; blockIdx.y is the slab.  Rows move as 16-byte
+// vectors: each thread takes kPermUnroll vectors kPermThreads apart (so a
+// warp's accesses stay contiguous within a row), reads all their table
+// entries, then all their sources, then writes, so that every thread keeps
+// kPermUnroll loads in flight against HBM.  Table entries outside [0, N) are
+// skipped.  I is the index type inside a slab (32-bit whenever N * vpr fits).
+constexpr int kPermThreads = 256;
+constexpr int kPermUnroll = 4;
+
+template <typename I>
+__global__ void __launch_bounds__(kPermThreads) permute_kernel(
+    const uint4* __restrict__ x, uint4* __restrict__ y, int32_t N, int32_t vpr,
+    const int32_t* __restrict__ perm, int inverse) {
   const int64_t slab = int64_t(blockIdx.y) * N * vpr;
-  const int64_t total = int64_t(N) * vpr;
-  for (int64_t t = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
-       t += int64_t(gridDim.x) * blockDim.x) {
-    const int32_t p = int32_t(t / vpr);
-    const int32_t v = int32_t(t - int64_t(p) * vpr);
-    const int32_t q = __ldg(perm + p);
-    if (uint32_t(q) >= uint32_t(N)) continue;
-    if (!inverse)
-      y[slab + int64_t(p) * vpr + v] = __ldg(x + slab + int64_t(q) * vpr + v);
-    else
-      y[slab + int64_t(q) * vpr + v] = __ldg(x + slab + int64_t(p) * vpr + v);
+  const uint4* __restrict__ xs = x + slab;
+  uint4* __restrict__ ys = y + slab;
+  const I total = I(N) * I(vpr);
+  const I base = I(blockIdx.x) * I(kPermThreads * kPermUnroll) + I(threadIdx.x);
+  I row[kPermUnroll], col[kPermUnroll];
+  int32_t q[kPermUnroll];
+#pragma unroll
+  for (int u = 0; u < kPermUnroll; ++u) {
+    const I e = base + I(u) * I(kPermThreads);
+    row[u] = e / I(vpr);
+    col[u] = e - row[u] * I(vpr);
+    q[u] = e < total ? __ldg(perm + row[u]) : -1;
+  }
+  uint4 val[kPermUnroll];
+#pragma unroll
+  for (int u = 0; u < kPermUnroll; ++u) {
+    if (uint32_t(q[u]) < uint32_t(N)) {
+      const I src = inverse ? row[u] : I(q[u]);
+      val[u] = __ldg(xs + src * I(vpr) + col[u]);
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kPermUnroll; ++u) {
+    if (uint32_t(q[u]) < uint32_t(N)) {
+      const I dst = inverse ? I(q[u]) : row[u];
+      ys[dst * I(vpr) + col[u]] = val[u];
+    }
   }
 }
 
@@ -205,12 +230,17 @@ cudaError_t launch_permute_rows(const void* x, void* y, int64_t BH, int32_t N, i
                                 const int32_t* perm, bool inverse, cudaStream_t s) {
   const int32_t vpr = row_bytes / 16;
   const int64_t total = int64_t(N) * vpr;
-  int64_t gx = cdiv(total, 256 * 4);
-  if (gx < 1) gx = 1;
-  if (gx > 65535) gx = 65535;
-  dim3 grid{unsigned(gx), unsigned(BH), 1u};
-  permute_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(x), static_cast<uint4*>(y), N,
-                                      vpr, perm, inverse ? 1 : 0);
+  const int64_t gx = cdiv(total, int64_t(kPermThreads) * kPermUnroll);
+  if (gx < 1 || gx > 0x7fffffff) return cudaErrorInvalidValue;
+  const dim3 grid{unsigned(gx), unsigned(BH), 1u};
+  const auto* xs = static_cast<const uint4*>(x);
+  auto* ys = static_cast<uint4*>(y);
+  // the last thread's index, base + (kPermUnroll - 1) * kPermThreads, stays
+  // below gx * kPermThreads * kPermUnroll <= total + kPermThreads * kPermUnroll
+  if (total + int64_t(kPermThreads) * kPermUnroll <= 0x7fffffffLL)
+    permute_kernel<int32_t><<<grid, kPermThreads, 0, s>>>(xs, ys, N, vpr, perm, inverse ? 1 : 0);
+  else
+    permute_kernel<int64_t><<<grid, kPermThreads, 0, s>>>(xs, ys, N, vpr, perm, inverse ? 1 : 0);
   return cudaGetLastError();
 }
 

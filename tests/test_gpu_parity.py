@@ -50,6 +50,45 @@ def test_permute_gathers_and_inverts_exactly(dtype, d):
     assert torch.equal(z, x)
 
 
+@pytest.mark.parametrize("dtype,d,N,BH", [(torch.float32, 12, 1000, (1, 1)),
+                                          (torch.bfloat16, 24, 333, (2, 5)),
+                                          (torch.float16, 8, 1, (1, 3)),
+                                          (torch.float32, 4, 70000, (1, 2))])
+def test_permute_odd_rows_and_ragged_lengths(dtype, d, N, BH):
+    """Rows of 3, 3, 1 and 1 vectors of 16 bytes, lengths that end inside a
+    CTA's chunk: every row lands where the table says, bit for bit."""
+    g = torch.Generator().manual_seed(N)
+    perm_np = torch.randperm(N, generator=g).numpy().astype(np.int32)
+    perm = torch.from_numpy(perm_np).to(dev())
+    x = torch.randn(*BH, N, d, device=dev()).to(dtype)
+    y, z = torch.empty_like(x), torch.empty_like(x)
+    fb.sparge_hilbert_permute(x, y, perm)
+    fb.sparge_inverse_permute(y, z, perm)
+    assert torch.equal(y, x[:, :, perm.long()])
+    assert torch.equal(z, x)
+
+
+def test_permute_skips_table_entries_outside_the_sequence():
+    N, d = 600, 64
+    perm_np = np.arange(N, dtype=np.int32)[::-1].copy()
+    perm_np[::7] = -1                     # rows whose entry is out of range
+    perm_np[3::11] = N + 5
+    perm = torch.from_numpy(perm_np).to(dev())
+    x = torch.randn(1, 2, N, d, device=dev()).to(torch.bfloat16)
+    y = torch.full_like(x, 7.0)
+    fb.sparge_hilbert_permute(x, y, perm)
+    ok = (perm_np >= 0) & (perm_np < N)
+    rows = np.nonzero(ok)[0]
+    assert torch.equal(y[:, :, rows], x[:, :, torch.from_numpy(perm_np[rows]).long().to(dev())])
+    assert bool((y[:, :, np.nonzero(~ok)[0]] == 7.0).all())
+    z = torch.full_like(x, -3.0)
+    fb.sparge_inverse_permute(x, z, perm)
+    tgt = torch.from_numpy(perm_np[rows]).long().to(dev())
+    assert torch.equal(z[:, :, tgt], x[:, :, rows])
+    untouched = np.setdiff1d(np.arange(N), perm_np[rows])
+    assert bool((z[:, :, untouched] == -3.0).all())
+
+
 # ----------------------------------------------------------------------------
 # stage 1: predictor
 # ----------------------------------------------------------------------------
