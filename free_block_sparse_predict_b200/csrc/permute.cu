@@ -10,6 +10,7 @@
 // exclusive scan over the survivors gives each grid token its rank.  The
 // gather / scatter kernels then move whole 16-byte chunks of token rows.
 #include <cstdint>
+#include <type_traits>
 
 #include "sparge_internal.h"
 
@@ -28,18 +29,26 @@ struct HilbertGrid {
   int64_t cube;     // 2^(n*bits)
 };
 
-// Curve position -> grid coordinates (transpose form, Gray decode, undo).
-__device__ __forceinline__ bool hilbert_decode(const HilbertGrid& g, int64_t h, int32_t* lin) {
-  uint32_t X[3] = {0, 0, 0};
-  for (int l = 0; l < g.bits; ++l)
-    for (int i = 0; i < g.n; ++i)
-      X[i] |= uint32_t((h >> (l * g.n + g.n - 1 - i)) & 1) << l;
-  uint32_t t = X[g.n - 1] >> 1;
-  for (int i = g.n - 1; i > 0; --i) X[i] ^= X[i - 1];
+// Curve position -> grid coordinates (transpose form, Gray decode, undo), for
+// a curve of NA axes: the axis loops unroll, so the coordinates stay in
+// registers.  h < 2^(NA * bits) <= 2^30.
+template <int NA>
+__device__ __forceinline__ bool hilbert_decode(const HilbertGrid& g, uint32_t h, int32_t* lin) {
+  uint32_t X[NA];
+#pragma unroll
+  for (int i = 0; i < NA; ++i) X[i] = 0;
+  for (int l = 0; l < g.bits; ++l) {
+#pragma unroll
+    for (int i = 0; i < NA; ++i) X[i] |= ((h >> (l * NA + NA - 1 - i)) & 1u) << l;
+  }
+  uint32_t t = X[NA - 1] >> 1;
+#pragma unroll
+  for (int i = NA - 1; i > 0; --i) X[i] ^= X[i - 1];
   X[0] ^= t;
   for (uint32_t Q = 2; Q != (1u << g.bits); Q <<= 1) {
     const uint32_t P = Q - 1;
-    for (int i = g.n - 1; i >= 0; --i) {
+#pragma unroll
+    for (int i = NA - 1; i >= 0; --i) {
       if (X[i] & Q) {
         X[0] ^= P;
       } else {
@@ -50,7 +59,8 @@ __device__ __forceinline__ bool hilbert_decode(const HilbertGrid& g, int64_t h, 
     }
   }
   int32_t L = 0;
-  for (int i = 0; i < g.n; ++i) {
+#pragma unroll
+  for (int i = 0; i < NA; ++i) {
     if (X[i] >= uint32_t(g.ext[i])) return false;
     L += int32_t(X[i]) * g.mul[i];
   }
@@ -58,13 +68,15 @@ __device__ __forceinline__ bool hilbert_decode(const HilbertGrid& g, int64_t h, 
   return true;
 }
 
+template <int NA>
 __global__ void hilbert_count_kernel(HilbertGrid g, int32_t* counts) {
   const int64_t base = int64_t(blockIdx.x) * kHilPerCta;
   int c = 0;
+#pragma unroll
   for (int k = 0; k < kHilPerThread; ++k) {
     const int64_t h = base + int64_t(threadIdx.x) * kHilPerThread + k;
     int32_t lin;
-    if (h < g.cube && hilbert_decode(g, h, &lin)) ++c;
+    if (h < g.cube && hilbert_decode<NA>(g, uint32_t(h), &lin)) ++c;
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xffffffffu, c, o);
@@ -78,6 +90,7 @@ __global__ void hilbert_count_kernel(HilbertGrid g, int32_t* counts) {
   }
 }
 
+template <int NA>
 __global__ void hilbert_scatter_kernel(HilbertGrid g, const int32_t* counts, int32_t ncount,
                                        int32_t N, int32_t prefix_len, int32_t L, int32_t* perm) {
   __shared__ int sh[kHilThreads / 32];
@@ -101,9 +114,10 @@ __global__ void hilbert_scatter_kernel(HilbertGrid g, const int32_t* counts, int
   int32_t lin[kHilPerThread];
   bool in[kHilPerThread];
   int c = 0;
+#pragma unroll
   for (int k = 0; k < kHilPerThread; ++k) {
     const int64_t h = base + k;
-    in[k] = h < g.cube && hilbert_decode(g, h, &lin[k]);
+    in[k] = h < g.cube && hilbert_decode<NA>(g, uint32_t(h), &lin[k]);
     c += in[k];
   }
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -119,6 +133,7 @@ __global__ void hilbert_scatter_kernel(HilbertGrid g, const int32_t* counts, int
   int warp_off = 0;
   for (int i = 0; i < w; ++i) warp_off += sh[i];
   int rank = s_base + warp_off + incl - c;
+#pragma unroll
   for (int k = 0; k < kHilPerThread; ++k) {
     if (in[k]) {
       if (rank < L) perm[prefix_len + rank] = prefix_len + lin[k];
@@ -213,17 +228,25 @@ cudaError_t launch_hilbert_index(int32_t N, int32_t prefix_len, int32_t T, int32
   int32_t* counts = static_cast<int32_t*>(ws);
   // a grid without an axis of extent > 1 has cube 0: the table is the identity
   const int64_t ctas = g.cube > 0 ? cdiv(g.cube, kHilPerCta) : 0;
-  if (ctas > 0) {
-    hilbert_count_kernel<<<unsigned(ctas), kHilThreads, 0, s>>>(g, counts);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
   const int64_t fill_ctas = cdiv(N, kHilThreads);
   int64_t grid = ctas > fill_ctas ? ctas : fill_ctas;
   if (grid < 1) grid = 1;
-  hilbert_scatter_kernel<<<unsigned(grid), kHilThreads, 0, s>>>(
-      g, counts, int32_t(ctas), N, prefix_len, g.cube > 0 ? L : 0, perm);
-  return cudaGetLastError();
+  const int32_t Lg = g.cube > 0 ? L : 0;
+  auto run = [&](auto na) -> cudaError_t {
+    constexpr int NA = decltype(na)::value;
+    if (ctas > 0) {
+      hilbert_count_kernel<NA><<<unsigned(ctas), kHilThreads, 0, s>>>(g, counts);
+      const cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+    hilbert_scatter_kernel<NA><<<unsigned(grid), kHilThreads, 0, s>>>(
+        g, counts, int32_t(ctas), N, prefix_len, Lg, perm);
+    return cudaGetLastError();
+  };
+  // a grid without an axis of extent > 1 launches no decode (cube 0)
+  if (g.n == 3) return run(std::integral_constant<int, 3>{});
+  if (g.n == 2) return run(std::integral_constant<int, 2>{});
+  return run(std::integral_constant<int, 1>{});
 }
 
 cudaError_t launch_permute_rows(const void* x, void* y, int64_t BH, int32_t N, int32_t row_bytes,
