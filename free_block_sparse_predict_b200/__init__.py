@@ -54,6 +54,49 @@ def _check(code: int) -> None:
         raise SpargeError(code, sparge_status_string(code))
 
 
+_TD = {SPARGE_F16: torch.float16, SPARGE_BF16: torch.bfloat16, SPARGE_F32: torch.float32}
+
+
+def _need(t, name: str, numel: int, dtype, device) -> None:
+    """The C ABI takes bare pointers and trusts the sizes that the parameters
+    imply; a tensor that is smaller, of another element type or on another
+    device would be read or written out of bounds, so it is refused here."""
+    if t is None:
+        return
+    if not t.is_cuda or t.device != device:
+        raise SpargeError(1, f"{name}: expected a tensor on {device}, got {t.device}")
+    if numel == 0:
+        return                      # an empty problem touches no memory
+    if dtype is not None and t.dtype != dtype:
+        raise SpargeError(1, f"{name}: expected {dtype}, got {t.dtype}")
+    if t.numel() < numel:
+        raise SpargeError(1, f"{name}: needs {numel} elements, has {t.numel()}")
+
+
+def _tiles(params):
+    B, Hq, Hkv = params.B, params.Hq, params.Hkv
+    Tm = -(-params.N // params.bq) if params.bq > 0 else 0
+    Tn = -(-params.N // params.bk) if params.bk > 0 else 0
+    return B, Hq, Hkv, Tm, Tn
+
+
+def _need_qk(params, q, k, v=None) -> None:
+    io = _TD.get(params.io_dtype)
+    dev = q.device
+    _need(q, "q", params.B * params.Hq * params.N * params.d, io, dev)
+    _need(k, "k", params.B * params.Hkv * params.N * params.d, io, dev)
+    _need(v, "v", params.B * params.Hkv * params.N * params.d, io, dev)
+
+
+def _need_mask(params, dev, mask=None, kv_idx=None, kv_cnt=None, s_q=None, s_k=None) -> None:
+    B, Hq, Hkv, Tm, Tn = _tiles(params)
+    _need(mask, "mask", B * Hq * Tm * Tn, torch.uint8, dev)
+    _need(kv_idx, "kv_idx", B * Hq * Tm * Tn, torch.int32, dev)
+    _need(kv_cnt, "kv_cnt", B * Hq * Tm, torch.int32, dev)
+    _need(s_q, "s_q", B * Hq * Tm, torch.float32, dev)
+    _need(s_k, "s_k", B * Hkv * Tn, torch.float32, dev)
+
+
 def make_params(B, Hq, Hkv, N, d, tau, theta, lam, causal=False, qk_int8=False,
                 io_dtype=torch.float16, o_dtype=None, scale=None, bq=128, bk=64) -> SpargeParams:
     """Hyper-parameters of one call: shapes, b_q/b_k, tau, theta, lambda, causal, INT8."""
@@ -76,6 +119,8 @@ def sparge_hilbert_workspace_bytes(T: int, Hg: int, Wg: int) -> int:
 
 
 def sparge_hilbert_index(N, prefix_len, T, Hg, Wg, perm, ws, stream=None) -> None:
+    _need(perm, "perm", max(int(N), 0), torch.int32, perm.device)
+    _need(ws, "ws", 0, None, perm.device)
     _check(lib().sparge_hilbert_index(N, prefix_len, T, Hg, Wg, _ptr(perm), _ptr(ws),
                                       ws.numel() * ws.element_size(), _stream(stream)))
 
@@ -84,6 +129,8 @@ def _perm_call(fn, src, dst, perm, stream):
     if src.dim() != 4 or src.shape != dst.shape or src.dtype != dst.dtype:
         raise SpargeError(1, "expected two [B, H, N, d] tensors of one shape and dtype")
     B, H, N, d = src.shape
+    _need(dst, "destination", 0, None, src.device)
+    _need(perm, "perm", N, torch.int32, src.device)
     _check(fn(_ptr(src), _ptr(dst), B, H, N, d, _DT[src.dtype], _ptr(perm), _stream(stream)))
 
 
@@ -98,6 +145,9 @@ def sparge_inverse_permute(y, x, perm, stream=None) -> None:
 
 
 def sparge_predict_mask(params, q, k, mask, kv_idx, kv_cnt, s_q, s_k, ws, stream=None) -> None:
+    _need_qk(params, q, k)
+    _need_mask(params, q.device, mask, kv_idx, kv_cnt, s_q, s_k)
+    _need(ws, "ws", 0, None, q.device)
     _check(lib().sparge_predict_mask(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(mask),
                                      _ptr(kv_idx), _ptr(kv_cnt), _ptr(s_q), _ptr(s_k), _ptr(ws),
                                      ws.numel() * ws.element_size(), _stream(stream)))
@@ -106,6 +156,8 @@ def sparge_predict_mask(params, q, k, mask, kv_idx, kv_cnt, s_q, s_k, ws, stream
 def sparge_predict_pool(params, q, k, ws, stream=None) -> None:
     """First half of sparge_predict_mask: block means, self-similarities and
     (qk_int8) the INT8 codes, written into ws."""
+    _need_qk(params, q, k)
+    _need(ws, "ws", 0, None, q.device)
     _check(lib().sparge_predict_pool(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(ws),
                                      ws.numel() * ws.element_size(), _stream(stream)))
 
@@ -113,6 +165,8 @@ def sparge_predict_pool(params, q, k, ws, stream=None) -> None:
 def sparge_predict_select(params, mask, kv_idx, kv_cnt, s_q, s_k, ws, stream=None) -> None:
     """Second half: the block mask and skip list from what sparge_predict_pool
     left in the same ws."""
+    _need(ws, "ws", 0, None, ws.device)
+    _need_mask(params, ws.device, mask, kv_idx, kv_cnt, s_q, s_k)
     _check(lib().sparge_predict_select(ctypes.byref(params), _ptr(mask), _ptr(kv_idx),
                                        _ptr(kv_cnt), _ptr(s_q), _ptr(s_k), _ptr(ws),
                                        ws.numel() * ws.element_size(), _stream(stream)))
@@ -124,17 +178,28 @@ def sparge_predict_mask_noalloc(params, q, k, mask, kv_idx, kv_cnt, s_q=None, s_
     allocate device memory when they call it.  The library's own static
     device scratch (32 MiB per GPU) holds the intermediates; calls that run
     concurrently on the GPU share it and race."""
+    _need_qk(params, q, k)
+    _need_mask(params, q.device, mask, kv_idx, kv_cnt, s_q, s_k)
     _check(lib().sparge_predict_mask_noalloc(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(mask),
                                              _ptr(kv_idx), _ptr(kv_cnt), _ptr(s_q), _ptr(s_k),
                                              _stream(stream)))
 
 
 def sparge_mask_compact(params, mask, kv_idx, kv_cnt, stream=None) -> None:
+    _need_mask(params, mask.device, mask, kv_idx, kv_cnt)
     _check(lib().sparge_mask_compact(ctypes.byref(params), _ptr(mask), _ptr(kv_idx),
                                      _ptr(kv_cnt), _stream(stream)))
 
 
 def sparge_attn_fwd(params, q, k, v, kv_idx, kv_cnt, o, ws, stats=None, stream=None) -> None:
+    _need_qk(params, q, k, v)
+    _need_mask(params, q.device, kv_idx=kv_idx, kv_cnt=kv_cnt)
+    _need(o, "o", params.B * params.Hq * params.N * params.d, _TD.get(params.o_dtype), q.device)
+    _need(ws, "ws", 0, None, q.device)
+    if stats is not None:
+        _need(stats, "stats", 0, None, q.device)
+        if stats.numel() * stats.element_size() < ctypes.sizeof(SpargeStats):
+            raise SpargeError(1, f"stats: needs {ctypes.sizeof(SpargeStats)} bytes")
     _check(lib().sparge_attn_fwd(ctypes.byref(params), _ptr(q), _ptr(k), _ptr(v), _ptr(kv_idx),
                                  _ptr(kv_cnt), _ptr(o), _ptr(ws), ws.numel() * ws.element_size(),
                                  _ptr(stats), _stream(stream)))

@@ -439,3 +439,45 @@ def test_empty_problems_are_no_ops():
         fb.sparge_attn_fwd(p, dummy, dummy, dummy, di, di, dummy, ws)
         fb.sparge_predict_mask(p, dummy, dummy, di, di, di, None, None, ws)
     torch.cuda.synchronize()
+
+
+def test_binding_refuses_buffers_the_parameters_do_not_fit():
+    """The C entry points take bare pointers; the binding checks every tensor
+    against the sizes, element types and device the parameters imply, so an
+    undersized or mistyped buffer raises instead of being read or written out
+    of bounds."""
+    w, t = workload("tiny")
+    p = params_for(w)
+    q, k, v = (to_dev(t[x], w.dtype) for x in ("q", "k", "v"))
+    ws = fb.workspace(p, dev())
+    mask, idx, cnt, s_q, s_k = fb.predict_outputs(p, dev())
+    o = torch.empty(q.shape, dtype=torch.float32, device=dev())     # o_dtype is f32 here
+    bad = [
+        # an fp16 O buffer for an f32 output would take half the bytes written
+        lambda: fb.sparge_attn_fwd(p, q, k, v, idx, cnt, torch.empty_like(q), ws),
+        lambda: fb.sparge_predict_mask(p, q[:, :, :10].contiguous(), k, mask, idx, cnt, None,
+                                       None, ws),
+        lambda: fb.sparge_predict_mask(p, q, k, mask[..., :1].contiguous(), idx, cnt, None, None,
+                                       ws),
+        lambda: fb.sparge_predict_mask(p, q, k, mask, idx.float(), cnt, None, None, ws),
+        lambda: fb.sparge_predict_mask(p, q.float(), k, mask, idx, cnt, None, None, ws),
+        lambda: fb.sparge_predict_select(p, mask, idx, cnt[..., :1].contiguous(), None, None, ws),
+        lambda: fb.sparge_attn_fwd(p, q, k, v[:, :, :5].contiguous(), idx, cnt, o, ws),
+        lambda: fb.sparge_attn_fwd(p, q, k, v, idx, cnt, o[:, :, :5].contiguous(), ws),
+        lambda: fb.sparge_attn_fwd(p, q, k, v, idx, cnt, o, ws,
+                                   torch.zeros(2, dtype=torch.int64, device=dev())),
+        lambda: fb.sparge_hilbert_permute(q, torch.empty_like(q),
+                                          torch.zeros(3, dtype=torch.int32, device=dev())),
+        lambda: fb.sparge_hilbert_permute(q, torch.empty_like(q),
+                                          torch.zeros(w.N, dtype=torch.int64, device=dev())),
+        lambda: fb.sparge_attn_fwd(p, q, k, v, idx, cnt, o.cpu(), ws),
+    ]
+    for call in bad:
+        with pytest.raises(fb.SpargeError) as e:
+            call()
+        assert e.value.code == 1
+    torch.cuda.synchronize()
+    # the well-formed call still runs
+    fb.sparge_predict_mask(p, q, k, mask, idx, cnt, s_q, s_k, ws)
+    fb.sparge_attn_fwd(p, q, k, v, idx, cnt, o, ws)
+    torch.cuda.synchronize()

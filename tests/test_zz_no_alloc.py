@@ -6,6 +6,8 @@ forbidden after start-up): its scratch is a static device array inside the
 library.  Its outputs must equal sparge_predict_mask's on the same inputs, on
 two calls in a row with different inputs (so stale scratch contents would
 show).  This file is collected last on purpose."""
+import ctypes
+
 import numpy as np
 import pytest
 import torch
@@ -57,9 +59,15 @@ def test_noalloc_rejects_what_it_cannot_hold():
     q, k = to_dev(t["q"], w.dtype), to_dev(t["k"], w.dtype)
     big = params_for(w.replace(N=131072, Hq=64, Hkv=8))   # pooled means exceed 32 MiB
     outs = fb.predict_outputs(params_for(w), dev())
+    # through the C entry point itself: the binding would refuse these
+    # tensors (smaller than the parameters imply) before the library saw them
+    P = lambda x: ctypes.c_void_p(x.data_ptr())
+    code = fb._native.lib().sparge_predict_mask_noalloc(ctypes.byref(big), P(q), P(k),
+                                                        *[P(x) for x in outs], None)
+    assert code == 5
     with pytest.raises(fb.SpargeError) as e:
         fb.sparge_predict_mask_noalloc(big, q, k, *outs)
-    assert e.value.code == 5
+    assert e.value.code == 1
     with pytest.raises(fb.SpargeError) as e:
         fb.sparge_predict_mask_noalloc(params_for(w, qk_int8=True), q, k, *outs)
     assert e.value.code == 2
