@@ -22,6 +22,7 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import glob
 import hashlib
 import json
 import os
@@ -41,7 +42,6 @@ from synth import get_workload, make_qkv  # noqa: E402
 
 METRIC = "sparse-attn dense-equiv TOPS at N=128K causal; sparsity; % tensor-core peak"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "attn_kernel_llm_128k.md")
 DATASHEET_BF16_TFLOPS = 2250.0
 L2_BYTES = 126e6  # B200 L2
 ATTN_SRC = os.path.join(ROOT, "free_block_sparse_predict_b200", "csrc", "attn_sm100.cu")
@@ -81,21 +81,25 @@ def load_peaks():
     return dict(PEAKS_FALLBACK), "fallback"
 
 
-def profiled_traffic(workload: str, seq_len: int, path: str = PROFILE_SUMMARY):
-    """dram bytes per attention launch from the committed ncu summary, if it
-    was taken on the current kernel source and on this workload and length."""
-    if not os.path.exists(path):
-        return None
-    text = open(path).read()
-    m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    h = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
-    wl = re.search(r"dram_bytes_workload:\s*(\S+)\s+N=(\d+)", text)
-    if not m or not h or not wl:
-        return None
-    if wl.group(1) != workload or int(wl.group(2)) != int(seq_len):
-        return None
+def profiled_traffic(workload: str, seq_len: int, path=None):
+    """dram bytes per attention launch from a committed ncu summary
+    (profiles/attn_kernel_*.md, or the one file given) taken on the current
+    kernel source and on this workload and length; None if there is none."""
+    paths = [path] if path else sorted(glob.glob(os.path.join(ROOT, "profiles",
+                                                             "attn_kernel_*.md")))
     cur = hashlib.sha256(open(ATTN_SRC, "rb").read()).hexdigest()
-    return float(m.group(1)) if h.group(1) == cur else None
+    for pth in paths:
+        if not os.path.exists(pth):
+            continue
+        text = open(pth).read()
+        m = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+        h = re.search(r"kernel_source_sha256:\s*([0-9a-f]+)", text)
+        wl = re.search(r"dram_bytes_workload:\s*(\S+)\s+N=(\d+)", text)
+        if not m or not h or not wl:
+            continue
+        if wl.group(1) == workload and int(wl.group(2)) == int(seq_len) and h.group(1) == cur:
+            return float(m.group(1))
+    return None
 
 
 def max_over_ranks(x: float, world: int, device=None) -> float:
