@@ -529,7 +529,7 @@ def _blas_threads():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(w, t, tiles_per_sample=32):
+def cpu_baseline(w, t, tiles_per_sample=64):
     ops, sec, n = _oracle_sample(w, t, tiles_per_sample)
     return {"value": round(ops / sec / 1e12, 9), "unit": "TOPS", "cores": _blas_threads(),
             "kind": "oracle",
@@ -717,7 +717,7 @@ def main():
                     help="override N of the workload (profiling a smaller case)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-tiles", type=int, default=32)
+    ap.add_argument("--cpu-tiles", type=int, default=64)
     ap.add_argument("--ref-tiles", type=int, default=4)
     ap.add_argument("--sweep", choices=("table6", "length", "tau", "permutation"), default=None,
                     help="run an ablation sweep instead of the benchmark (one JSON line per point)")
