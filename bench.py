@@ -354,6 +354,38 @@ def run_native(args, rank, world, local_rank):
                "d2h_bytes_per_step": nb(o), "ms_per_step": round(e2e_ms / args.steps, 3),
                "pipelined": "H2D of step s+1 and D2H of step s overlap the compute of step s"}
 
+    # ---- optional: the same step captured once into a CUDA graph and replayed
+    graph_line = None
+    if args.graph:
+        from free_block_sparse_predict_b200.graph import SpargeGraph
+        g = SpargeGraph(p, grid=(w.prefix_len, *w.grid) if w.grid else None, device=dev)
+        g.q.copy_(q)
+        g.k.copy_(k)
+        g.v.copy_(v)
+        for _ in range(args.warmup):
+            g.run()
+        torch.cuda.synchronize()
+        gspan = [(ev(), ev()) for _ in range(args.steps)]
+        g0, g1 = ev(), ev()
+        g0.record(stream)
+        for s_ in range(args.steps):
+            if flush is not None:
+                flush.fill_(s_ & 255)
+                flush_rd.max()
+            gspan[s_][0].record(stream)
+            g.run()
+            gspan[s_][1].record(stream)
+        g1.record(stream)
+        torch.cuda.synchronize()
+        g_ms = (g0.elapsed_time(g1) if flush is None
+                else float(sum(a.elapsed_time(b) for a, b in gspan)))
+        g_ms = max_over_ranks(g_ms, world, dev)
+        graph_line = {"value": round(aggregate_tops(world, dense_equiv_ops(w), args.steps, g_ms), 3),
+                      "unit": "TOPS", "ms_per_step": round(g_ms / args.steps, 4),
+                      "what": "the same step (permutes, predictor, attention) captured once "
+                              "into a CUDA graph and replayed"}
+        del g
+
     if rank != 0:
         return None
 
@@ -442,6 +474,7 @@ def run_native(args, rank, world, local_rank):
                           + pv_blocks * blk_flops) / (peak * 1e12) / (attn_ms * 1e-3), 4),
                      "kernel": "attn_kernel (tcgen05), issued MMA flops per launch / launch time"},
         "gpu_launches": launches_per_step * args.steps,
+        **({"graph": graph_line} if graph_line else {}),
         "clocks": clocks,
         "e2e": e2e,
     }
@@ -716,6 +749,8 @@ def main():
     ap.add_argument("--seq-len", type=int, default=0,
                     help="override N of the workload (profiling a smaller case)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="also time the step captured into a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-tiles", type=int, default=64)
     ap.add_argument("--ref-tiles", type=int, default=4)
