@@ -426,6 +426,18 @@ def test_quantize_blocks_reconstruction_bound_and_extremes():
     assert dz[0] == 0 and not z.any()
 
 
+def test_quantize_blocks_rounds_ties_to_even():
+    """With absmax 127 the multiplier 127/absmax is exactly 1, so x * inv is
+    x itself: halves must go to the even neighbour (2.5 -> 2, 3.5 -> 4,
+    -2.5 -> -2, 126.5 -> 126), which a round-half-away or floor(x + 0.5)
+    reading would get wrong."""
+    X = np.zeros((64, 8), np.float32)
+    X[0, :8] = [127.0, 2.5, 3.5, -2.5, -3.5, 126.5, 0.5, -0.5]
+    codes, delta = orc.quantize_blocks(X, 64)
+    assert delta[0] == np.float32(1.0)
+    assert codes[0].tolist() == [127, 2, 4, -2, -4, 126, 0, 0]
+
+
 def test_k_smoothing_leaves_exact_attention_unchanged():
     # subtracting kbar shifts every score row by q.kbar: softmax is invariant
     N, d = 200, 16
