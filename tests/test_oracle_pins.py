@@ -249,6 +249,30 @@ def test_fix_rule_theta_below_minus_one_is_pure_topcdf():
     assert pr["M"].sum() < pr["M"].size
 
 
+def test_theta_comparisons_are_strict():
+    """Eq. 7 and Eq. 9 compare with a strict "<": a K block whose
+    self-similarity equals theta keeps a finite S_hat column and is not forced
+    on; blocks below theta are -inf in S_hat and forced on in M."""
+    rng = np.random.default_rng(77)
+    K = rng.standard_normal((1, 1, 512, 16))
+    # self-similar query blocks (s_q near 1), so no row is a fix row
+    Q = (np.repeat(rng.standard_normal((4, 16)), 128, axis=0)
+         + 0.01 * rng.standard_normal((512, 16)))[None, None]
+    sk = orc.predict_mask(Q, K, 128, 64, 0.3, -2.0, False, 0.25)["s_k"][0, 0]
+    j0 = int(np.argsort(sk)[len(sk) // 2])
+    theta = float(sk[j0])
+    pr = orc.predict_mask(Q, K, 128, 64, 0.3, theta, False, 0.25)
+    S, M = pr["S_hat"][0, 0], pr["M"][0, 0]
+    below = sk < theta
+    assert not below[j0] and below.any() and (~below).sum() >= 2
+    assert np.isfinite(S[:, ~below]).all() and np.isneginf(S[:, below]).all()
+    assert (pr["s_q"][0, 0] >= theta).all()
+    for i in range(S.shape[0]):
+        keep, _, _ = orc.topcdf(orc.row_softmax(S[i]), 0.3)
+        assert np.array_equal(M[i], keep | below)
+    assert not M[:, j0].all()          # the data tell a forced column from a kept one
+
+
 def test_fix_rule_rows_and_columns():
     vis = np.ones((3, 4), dtype=bool)
     M = np.zeros((3, 4), dtype=bool)
