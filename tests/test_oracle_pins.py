@@ -416,6 +416,11 @@ def test_lambda_decision_is_per_warp_slice_and_order_dependent():
     idx_r[0, 0, 0, :2] = [1, 0]
     _, st_r = orc.sparse_attention(Q, K, V, idx_r, cnt, 128, 64, -1.0, False, 1.0)
     assert st_r["skipped_slices"] == 1 and st_r["pv_slices"] == 7
+    # Eq. 3's test is strict: slices exactly lambda = -8 below their max are kept
+    _, st_eq = orc.sparse_attention(Q, K, V, idx, cnt, 128, 64, -8.0, False, 1.0)
+    assert st_eq["skipped_slices"] == 0 and st_eq["pv_slices"] == 8
+    _, st_lt = orc.sparse_attention(Q, K, V, idx, cnt, 128, 64, -7.999, False, 1.0)
+    assert st_lt["skipped_slices"] == 3
 
 
 def test_row_with_no_visible_key_outputs_zero():
