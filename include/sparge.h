@@ -102,13 +102,18 @@ sparge_status_t sparge_hilbert_index(int32_t N, int32_t prefix_len, int32_t T, i
                                      cudaStream_t stream);
 
 /* y[b, h, p, :] = x[b, h, perm[p], :] for x, y [B, H, N, d] of dtype (16-bit
- * or f32).  perm is a device permutation of 0..N-1 (e.g. from
- * sparge_hilbert_index); x and y must not overlap. */
+ * or f32).  perm is a device array of N int32 entries, normally a
+ * permutation of 0..N-1 (e.g. from sparge_hilbert_index); a row whose entry
+ * lies outside [0, N) is skipped (y's row is left as it was).  x and y must
+ * not overlap (SPARGE_EINVAL).  A row of d elements must be a multiple of 16
+ * bytes and B * H at most 65535 (SPARGE_EUNSUPPORTED otherwise); B, H or
+ * N = 0 is a no-op.  HBM-bound: each row is read once and written once. */
 sparge_status_t sparge_hilbert_permute(const void* x, void* y, int32_t B, int32_t H, int32_t N,
                                        int32_t d, sparge_dtype_t dtype, const int32_t* perm,
                                        cudaStream_t stream);
 
-/* The inverse: x[b, h, perm[p], :] = y[b, h, p, :]. */
+/* The inverse: x[b, h, perm[p], :] = y[b, h, p, :], under the same rules (a
+ * row whose entry lies outside [0, N) is not written). */
 sparge_status_t sparge_inverse_permute(const void* y, void* x, int32_t B, int32_t H, int32_t N,
                                        int32_t d, sparge_dtype_t dtype, const int32_t* perm,
                                        cudaStream_t stream);
