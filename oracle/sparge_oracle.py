@@ -39,13 +39,13 @@ design notes):
       row whose m_local is -inf contributes -inf.  rowsum(P~) always enters l.
   R7  A row with l = 0 outputs 0.
   R8  GQA: query head h reads KV head h // (Hq/Hkv).
-  R9  INT8: kbar = per-(batch, KV head) float32 mean of K over all tokens;
-      K' = K - kbar in float32; per block delta = absmax/127 (the dequantisation
-      scale) and inv = 127/absmax, both float32 divides; code =
-      round-half-even(x * inv) with a float32 multiply, clamped to +-127.
-      The subtracted kbar shifts each score row by a constant, so no bias term
-      ("delta Bias" of Algorithm 1 step 10) is added.  The predictor itself
-      pools the original K.
+  R9  INT8: kbar = per-(batch, KV head) mean of K over all tokens, taken in
+      float64 and rounded once to float32; K' = K - kbar in float32; per block
+      delta = absmax/127 (the dequantisation scale, an IEEE float32 divide);
+      code = round-half-even(x / delta) of the IEEE float32 quotient, clamped
+      to +-127; delta = 0 gives all-zero codes.  The subtracted kbar shifts
+      each score row by a constant, so no bias term ("delta Bias" of
+      Algorithm 1 step 10) is added.  The predictor itself pools the original K.
 """
 from __future__ import annotations
 
@@ -296,8 +296,14 @@ def predict_mask(Q: np.ndarray, K: np.ndarray, bq: int, bk: int, tau: float, the
                 keep, t_star, cb = topcdf(P[fin], tau)
                 Mt[i, fin] = keep
                 if tau < 1.0:
+                    # a cumulative mass within amb_cum of the cut can land on
+                    # either side of tau in float32
                     near_cut = np.abs(cb - tau) <= amb_cum
-                    near_tie = np.abs(P[fin] - t_star) <= amb_tie * t_star
+                    # two near-equal weights on opposite sides of the cut can
+                    # swap places in float32; a weight alone at t_star cannot
+                    pf = P[fin]
+                    band = np.abs(pf - t_star) <= amb_tie * t_star
+                    near_tie = band if (band & ~keep).any() else np.zeros_like(band)
                     a = amb[b, h, i]
                     a[np.flatnonzero(fin)[near_cut | near_tie]] = True
             # an entry whose column is near theta can flip in or out of TopCdf
@@ -343,12 +349,16 @@ def mask_statistics(M: np.ndarray, s_q: np.ndarray, s_k: np.ndarray, theta: floa
 # ============================================================================
 
 def k_smooth_mean(K32: np.ndarray) -> np.ndarray:
-    """Per-(batch, head) float32 mean of K over all tokens.  K32 [B,H,N,d] float32."""
+    """Per-(batch, head) mean of K over all tokens (Algorithm 1 step 2's
+    smoothing), summed in float64 and rounded once to float32.
+    K32 [B,H,N,d] float32."""
     return K32.astype(np.float64).mean(axis=2).astype(np.float32)
 
 
 def quantize_blocks(X32: np.ndarray, b: int):
-    """Per-block symmetric INT8 of X32 [N, d] float32 (reading R9).
+    """Per-block symmetric INT8 of X32 [N, d] float32 (reading R9): delta =
+    absmax / 127 and code = rint(x / delta), both IEEE float32 divides, the
+    quotient rounded half to even.
 
     Returns (codes int8 [N, d], delta float32 [T])."""
     N = X32.shape[0]
@@ -360,9 +370,8 @@ def quantize_blocks(X32: np.ndarray, b: int):
         blk = X32[r0:r1]
         amax = np.float32(np.abs(blk).max()) if blk.size else np.float32(0)
         delta[i] = np.float32(amax / np.float32(127.0))
-        if amax > 0:
-            inv = np.float32(np.float32(127.0) / amax)
-            v = np.rint(blk * inv)         # float32 multiply, round half to even
+        if delta[i] > 0:
+            v = np.rint(blk / delta[i])    # float32 quotient, round half to even
             codes[r0:r1] = np.clip(v, -127, 127).astype(np.int8)
     return codes, delta
 

@@ -528,3 +528,205 @@ def test_compressed_scores_equal_token_scores_for_constant_blocks():
     S = d ** -0.5 * Q[0, 0] @ K[0, 0].T
     assert np.allclose(pr["S_hat"][0, 0], S[::128, ::64], atol=1e-12)
     assert np.allclose(pr["s_q"], 1.0) and np.allclose(pr["s_k"], 1.0)
+
+
+# ----------------------------------------------------------------------------
+# pins added for steps a plausible slip could break without any pin above
+# noticing: the softmax of Algorithm 1 step 5, Eq. 9's strict row test, the K
+# smoothing of Algorithm 1 step 2, the INT8 quotient, and the ambiguity map
+# ----------------------------------------------------------------------------
+
+def _constant_block_inputs(shat_row, n_q=192, d=4):
+    """Q and K whose blocks are constant tokens, so that S_hat[i, j] equals
+    the given values for every query block i (Eq. 4-7 with identical tokens:
+    the block mean is the token itself and its self-similarity is 1).
+    With d = 4 the scale is 1/2; q = (2, 0, 0, 0) and k_j = (v_j, 0, 0, 0)
+    give scale * q . k_j = v_j."""
+    Tn = len(shat_row)
+    N = max(n_q, 64 * Tn)
+    Q = np.zeros((1, 1, N, d))
+    Q[..., 0] = 2.0
+    K = np.zeros((1, 1, N, d))
+    K[..., 1] = 1.0                         # keys past the listed blocks: some token
+    for j, v in enumerate(shat_row):
+        K[0, 0, 64 * j:64 * (j + 1), 0] = v
+        K[0, 0, 64 * j:64 * (j + 1), 1] = 0.0
+    return Q, K, N
+
+
+def test_row_softmax_hand_worked():
+    # S_hat = (ln 5, ln 3, ln 2) + c: the softmax is (5, 3, 2) / 10 whatever c
+    for c in (0.0, 7.25, -40.0):
+        P = orc.row_softmax(np.log([5.0, 3.0, 2.0]) + c)
+        assert np.allclose(P, [0.5, 0.3, 0.2], rtol=0, atol=1e-14)
+    # -inf entries get weight 0 and leave the others' ratio alone
+    P = orc.row_softmax(np.array([np.log(3.0), -np.inf, 0.0, -np.inf]))
+    assert np.allclose(P, [0.75, 0.0, 0.25, 0.0], rtol=0, atol=1e-14)
+    assert np.all(orc.row_softmax(np.full(3, -np.inf)) == 0)
+
+
+@pytest.mark.parametrize("tau,keep", [(0.45, [0]), (0.6, [0, 1]), (0.85, [0, 1, 2])])
+def test_predicted_row_from_hand_worked_shat(tau, keep):
+    """Constant blocks give S_hat = (ln 5, ln 3, ln 2) + 1.5 on every query
+    row, so P_hat = (0.5, 0.3, 0.2) and TopCdf(tau) keeps {0} at tau = 0.45,
+    {0, 1} at 0.6 and all three at 0.85 (Eq. 7, 8).  A softmax at another
+    temperature (e.g. exp(2 S)) gives (0.66, 0.24, 0.11) and keeps {0} at 0.6."""
+    row = np.log([5.0, 3.0, 2.0]) + 1.5
+    Q, K, N = _constant_block_inputs(row)
+    pr = orc.predict_mask(Q, K, 128, 64, tau, 0.5, False, 0.5)
+    assert np.allclose(pr["S_hat"][0, 0, :, :3], row, atol=1e-12)
+    assert np.allclose(pr["s_q"], 1.0) and np.allclose(pr["s_k"][0, 0, :3], 1.0)
+    for i in range(pr["M"].shape[2]):
+        assert np.flatnonzero(pr["M"][0, 0, i, :3]).tolist() == keep
+        assert not pr["amb"][0, 0, i].any()
+
+
+def test_fix_rule_row_test_is_strict():
+    """Eq. 9 forces the rows of query blocks with s_q < theta: a row whose
+    self-similarity is exactly theta is not a fix row, one just below is."""
+    theta = 0.5
+    vis = np.ones((3, 4), dtype=bool)
+    s_q = np.array([theta, np.nextafter(theta, -1.0), theta + 0.25])
+    out = orc.apply_fix_rule(np.zeros((3, 4), dtype=bool), s_q, np.full(4, 0.9), theta, vis)
+    assert out.sum(axis=1).tolist() == [0, 4, 0]
+    # and through the whole predictor: a query block with s_q exactly theta
+    rng = np.random.default_rng(11)
+    Q = rng.standard_normal((1, 1, 512, 16))
+    K = (np.repeat(rng.standard_normal((8, 16)), 64, axis=0)
+         + 0.01 * rng.standard_normal((512, 16)))[None, None]       # s_k near 1
+    sq = orc.predict_mask(Q, K, 128, 64, 0.3, -2.0, False, 0.25)["s_q"][0, 0]
+    i0 = int(np.argmax(sq))
+    pr = orc.predict_mask(Q, K, 128, 64, 0.3, float(sq[i0]), False, 0.25)
+    M = pr["M"][0, 0]
+    assert (pr["s_k"] >= sq[i0]).all()                               # no fix column
+    keep, _, _ = orc.topcdf(orc.row_softmax(pr["S_hat"][0, 0, i0]), 0.3)
+    assert np.array_equal(M[i0], keep) and not M[i0].all()
+    below = sq < sq[i0]
+    assert below.any() and M[below].all()
+
+
+def test_k_smoothing_mean_hand_value_and_offset_invariance():
+    """Algorithm 1 step 2 subtracts the per-head mean of K over all tokens
+    before the per-block INT8 of K.  On dyadic inputs every step is exact, so
+    kbar equals the rational mean and adding any per-channel constant c to K
+    leaves K - kbar, and therefore every code and scale, unchanged."""
+    from fractions import Fraction
+    rng = np.random.default_rng(5)
+    N, d = 256, 8
+    K = (rng.integers(-40, 41, size=(1, 1, N, d)) / 8.0).astype(np.float32)
+    K[0, 0, :, 3] += 5.0
+    want = [Fraction(0)] * d
+    for n in range(N):
+        for c in range(d):
+            want[c] += Fraction(float(K[0, 0, n, c]))
+    want = [w / N for w in want]
+    Q = rng.standard_normal((1, 2, N, d)).astype(np.float32)
+    qt = orc.quantize_qk(Q, K, 128, 64)
+    assert [Fraction(float(v)) for v in qt["kbar"][0, 0]] == want
+    off = (64.0 * (1 + np.arange(d))).astype(np.float32)
+    qt2 = orc.quantize_qk(Q, K + off, 128, 64)
+    assert np.array_equal(qt2["kbar"][0, 0], qt["kbar"][0, 0] + off)
+    assert np.array_equal(qt2["k_codes"], qt["k_codes"])
+    assert np.array_equal(qt2["dk"], qt["dk"])
+    assert (qt["k_codes"] != 0).any()
+
+
+def _f32_round(q):
+    """Round a rational to the nearest float32, ties to even (IEEE 754),
+    by exact integer arithmetic on the significand."""
+    from fractions import Fraction
+    if q == 0:
+        return Fraction(0)
+    sgn = -1 if q < 0 else 1
+    a = abs(q)
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    e = max(e, -126)                      # subnormals keep the bottom exponent
+    ulp = Fraction(2) ** (e - 23)
+    m = round(a / ulp)                    # Python rounds Fractions half to even
+    return sgn * m * ulp
+
+
+def _exact_int8_code(x, delta):
+    """rint of the correctly rounded float32 quotient x / delta, clamped."""
+    from fractions import Fraction
+    if delta == 0:
+        return 0
+    v = round(_f32_round(Fraction(float(x)) / Fraction(float(delta))))
+    return max(-127, min(127, v))
+
+
+# (absmax, x) float32 pairs whose float32 quotient x / (absmax / 127) rounds to
+# one integer while x * (127 / absmax) rounds to the next: they tell the
+# division of reading R9 from a multiply by the reciprocal
+_QUOTIENT_CASES = [(2.408083438873291, -2.28483510017395),
+                   (7.719466686248779, -6.534193992614746),
+                   (7.485044002532959, -5.5106425285339355),
+                   (7.883794784545898, 5.617980003356934),
+                   (3.9020028114318848, 2.842010021209717),
+                   (3.9020028114318848, 3.149254322052002)]
+
+
+def test_int8_codes_are_rint_of_the_float32_quotient():
+    """Reading R9: delta = fl32(absmax / 127) and code = rint(fl32(x / delta)).
+    Checked against exact rational arithmetic: on crafted blocks where the
+    quotient and the product with the reciprocal round to different integers,
+    and on random blocks."""
+    from fractions import Fraction
+    for amax, x in _QUOTIENT_CASES:
+        blk = np.zeros((64, 4), np.float32)
+        blk[0, 0] = np.float32(amax)
+        blk[1, 1] = np.float32(x)
+        codes, delta = orc.quantize_blocks(blk, 64)
+        assert Fraction(float(delta[0])) == _f32_round(Fraction(float(np.float32(amax))) / 127)
+        assert int(codes[1, 1]) == _exact_int8_code(np.float32(x), delta[0])
+        assert int(codes[0, 0]) == 127
+    X = (RNG.standard_normal((128, 16)) * 2.5).astype(np.float32)
+    codes, delta = orc.quantize_blocks(X, 64)
+    for i in range(2):
+        for r in range(64):
+            for c in range(16):
+                assert int(codes[64 * i + r, c]) == _exact_int8_code(X[64 * i + r, c], delta[i])
+
+
+def test_ambiguity_map_flags_only_decisions_near_the_cut():
+    """Entries are ambiguous when the normalised mass before them is within
+    1e-4 of tau, or when near-equal weights sit on both sides of the cut.
+    P_hat = (0.5, 0.3, 0.2): at tau = 0.5 + 5e-5 the second entry (mass 0.5
+    before it) is flagged; at tau = 0.5 + 1e-3 nothing is."""
+    row = np.log([5.0, 3.0, 2.0]) + 1.5
+    Q, K, N = _constant_block_inputs(row)
+    pr = orc.predict_mask(Q, K, 128, 64, 0.5 + 5e-5, 0.5, False, 0.5)
+    assert pr["amb"][0, 0, :, :3].tolist() == [[False, True, False]] * 2
+    pr = orc.predict_mask(Q, K, 128, 64, 0.5 + 1e-3, 0.5, False, 0.5)
+    assert not pr["amb"].any()
+    assert pr["M"][0, 0, :, :3].tolist() == [[True, True, False]] * 2
+    # weights 4 : 3 : 3(1 - 5e-6) : 1 at tau = 0.5: the cut falls between the
+    # two near-equal weights, so both are flagged and nothing else
+    row = np.log([4.0, 3.0, 3.0 * (1 - 5e-6), 1.0]) + 1.5     # no zero key token
+    Q, K, N = _constant_block_inputs(row)
+    pr = orc.predict_mask(Q, K, 128, 64, 0.5, 0.5, False, 0.5)
+    assert pr["amb"][0, 0, 0, :4].tolist() == [False, True, True, False]
+    assert pr["M"][0, 0, 0, :4].tolist() == [True, True, False, False]
+    # a weight alone at the cut is not ambiguous
+    row = np.log([4.0, 3.0, 2.0, 1.0]) + 1.5
+    Q, K, N = _constant_block_inputs(row)
+    pr = orc.predict_mask(Q, K, 128, 64, 0.5, 0.5, False, 0.5)
+    assert not pr["amb"].any()
+
+
+def test_whole_forward_dense_limit_with_permutation_equals_softmax_attention():
+    """sparge_forward chains permute -> predict -> attention -> inverse.  With
+    theta > 1 (every block a fix block) and lambda = -inf, and with or without
+    the Hilbert permutation (dense attention is permutation invariant, rebuttal
+    page, reply to Weakness 3.2), it is plain softmax attention."""
+    N, P, grid, d = 300, 12, (2, 8, 9), 16
+    perm = orc.hilbert_permutation(N, P, *grid)
+    Q, K, V = rand_qkv(1, 4, 2, N, d)
+    ref = dense_attention(Q, K, V, d ** -0.5)
+    for pm in (None, perm):
+        O, pred, st = orc.sparge_forward(Q, K, V, 128, 64, 0.9, 1.5, -np.inf, False, d ** -0.5,
+                                         perm=pm)
+        assert np.allclose(O, ref, atol=1e-12)
+        assert pred["M"].all() and st["skipped_slices"] == 0
