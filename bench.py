@@ -54,17 +54,52 @@ def dense_equiv_ops(w) -> float:
 
 def pool_bytes(w) -> float:
     """Algorithmic HBM bytes of one predictor pooling stage: one read of Q and
-    K, the block means and self-similarities written, and with INT8 the Q codes,
-    k-bar (from the K means), a second read of K and the K codes."""
+    K, the block means and self-similarities written, and with INT8 the codes
+    of Q and K and their block scales."""
     es = 2
     Tm, Tn = -(-w.N // w.bq), -(-w.N // w.bk)
     bq_, bk_ = w.B * w.Hq, w.B * w.Hkv
     b = (bq_ + bk_) * w.N * w.d * es + (bq_ * Tm + bk_ * Tn) * (w.d + 1) * 4
     if w.qk_int8:
         b += bq_ * w.N * w.d + bq_ * Tm * 4                       # Q codes, scales
-        b += bk_ * Tn * w.d * 4                                   # k-bar from the K means
-        b += bk_ * w.N * w.d * es + bk_ * w.N * w.d + bk_ * Tn * 4  # K again, codes, scales
+        b += bk_ * w.N * w.d + bk_ * Tn * 4                       # K codes, scales
     return float(b)
+
+
+def pool_extra_bytes(w) -> float:
+    """Bytes the INT8 pooling stage moves beyond the algorithmic ones: the
+    second read of K (the codes of K - kbar need kbar, a mean over all of K)
+    and the float64 block sums that kbar is reduced from."""
+    if not w.qk_int8:
+        return 0.0
+    Tn = -(-w.N // w.bk)
+    bk_ = w.B * w.Hkv
+    return float(bk_ * w.N * w.d * 2 + 2 * bk_ * Tn * w.d * 8)
+
+
+def attn_peak_tflops(w, peaks, qk_blocks, pv_blocks, key="bf16_tflops_sustained"):
+    """The tensor peak for the attention kernel's own mix of contractions: Q K^T
+    in INT8 (twice the measured bf16 rate, the nominal dense ratio of the two)
+    or in the I/O dtype, P~V in fp16 (the bf16 rate).  The flop-weighted
+    harmonic mean: issued flops over the time they need at those peaks."""
+    bf = float(peaks[key])
+    qk_peak = 2.0 * bf if w.qk_int8 else bf
+    tot = qk_blocks + pv_blocks
+    if tot == 0:
+        return bf
+    return tot / (qk_blocks / qk_peak + pv_blocks / bf)
+
+
+def workload_config(w, world, t_bytes):
+    """The config object of the JSON line, shared by both arms."""
+    return {"workload": f"{w.name}: B{w.B} Hq{w.Hq} Hkv{w.Hkv} N{w.N} d{w.d} "
+                        f"{w.dtype} causal={int(w.causal)} int8_qk={int(w.qk_int8)} "
+                        f"tau={w.tau} theta={w.theta} lambda={w.lam}",
+            "global_batch": w.B * world, "seq_len": w.N,
+            "parallelism": f"replicas x{world}",
+            "l2": "inputs larger than L2 (no flush)" if t_bytes > L2_BYTES
+            else "inputs fit in L2: 256 MB rewritten, then 256 MB read, between "
+                 "steps; steps timed alone"}
 
 
 def fp32_peak_tflops(peaks) -> float:
@@ -211,8 +246,9 @@ def run_native(args, rank, world, local_rank):
 
     launches_per_step = 0
 
-    def step(qs, ks, vs, os_, timing=None):
+    def step(qs, ks, vs, os_, timing=None, prm=None):
         nonlocal launches_per_step
+        prm = p if prm is None else prm
         n = 0
         if w.grid:
             fb.sparge_hilbert_index(w.N, w.prefix_len, *w.grid, perm, hws, stream)
@@ -225,15 +261,15 @@ def run_native(args, rank, world, local_rank):
             dst = os_
         if timing:
             timing[0].record(stream)
-        fb.sparge_predict_pool(p, qs, ks, ws, stream)
-        n += 4 if w.qk_int8 else 1
+        fb.sparge_predict_pool(prm, qs, ks, ws, stream)
+        n += 5 if w.qk_int8 else 1
         if timing:
             timing[1].record(stream)
-        fb.sparge_predict_select(p, mask, idx, cnt, None, None, ws, stream)
+        fb.sparge_predict_select(prm, mask, idx, cnt, None, None, ws, stream)
         n += 1
         if timing:
             timing[2].record(stream)
-        fb.sparge_attn_fwd(p, qs, ks, vs, idx, cnt, dst, ws, stats, stream)
+        fb.sparge_attn_fwd(prm, qs, ks, vs, idx, cnt, dst, ws, stats, stream)
         n += 2 if w.dtype == "bf16" else 1
         if timing:
             timing[3].record(stream)
@@ -256,6 +292,7 @@ def run_native(args, rank, world, local_rank):
     st = stats.cpu().numpy().astype(np.int64)
     if fb.sparge_device_status(ws) != 0:
         raise RuntimeError("device status reported an error")
+    mask_h0 = mask[:, 0].cpu().numpy().astype(bool) if rank == 0 else None
 
     sampler = ClockSampler(_gpu_uuid(torch, dev)) if local_rank == 0 or world > 1 else None
     barrier()
@@ -301,6 +338,51 @@ def run_native(args, rank, world, local_rank):
     ms_step = ms_total / args.steps
     ops_step = dense_equiv_ops(w)
     value = aggregate_tops(world, ops_step, args.steps, ms_total)
+
+    # ---- the same workload in a sparse regime: theta = -1 makes every block
+    # selective and tau = 0.5 lets TopCdf drop blocks, so the skipping of Eq. 2
+    # is what gets timed.  Reported beside the headline, never instead of it.
+    sparse = None
+    if not args.no_sparse_regime:
+        ps = fb.make_params(w.B, w.Hq, w.Hkv, w.N, w.d, 0.5, -1.0, w.lam, causal=w.causal,
+                            qk_int8=w.qk_int8, io_dtype=tdt)
+        for _ in range(args.warmup):
+            step(q, k, v, o, prm=ps)
+        torch.cuda.synchronize()
+        stats.zero_()
+        step(q, k, v, o, prm=ps)
+        torch.cuda.synchronize()
+        sst = [int(x) for x in stats.cpu()]
+        sper = [(ev(), ev(), ev(), ev()) for _ in range(args.steps)]
+        sspan = [(ev(), ev()) for _ in range(args.steps)]
+        for s_ in range(args.steps):
+            if flush is not None:
+                flush.fill_(s_ & 255)
+                flush_rd.max()
+            sspan[s_][0].record(stream)
+            step(q, k, v, o, sper[s_], prm=ps)
+            sspan[s_][1].record(stream)
+        torch.cuda.synchronize()
+        if fb.sparge_device_status(ws) != 0:
+            raise RuntimeError("device status reported an error")
+        s_step = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in sspan])), world, dev)
+        s_attn = float(np.mean([a.elapsed_time(b) for (_, _, a, b) in sper]))
+        s_pred = float(np.mean([a.elapsed_time(c) for (a, _, c, _) in sper]))
+        vis = _visible_blocks(w)
+        sparse = {
+            "tau": 0.5, "theta": -1.0, "lambda": w.lam, "steps": args.steps,
+            "value": round(aggregate_tops(world, dense_equiv_ops(w), 1, s_step), 3), "unit": "TOPS",
+            "latency_ms": {"step": round(s_step, 4), "predict": round(s_pred, 4),
+                           "attention": round(s_attn, 4)},
+            "sparsity": {"mg": round(1.0 - sst[1] / vis, 6),
+                         "pv_slices_skipped": round(sst[4] / max(1, sst[3] + sst[4]), 6),
+                         "total": round(1.0 - (sst[1] + sst[3] / 4.0) / (2.0 * vis), 6)},
+            "work": {"qk_blocks": sst[1], "pv_blocks": sst[2], "visible_blocks": vis},
+            "attention_tflops": round((sst[1] + sst[2]) * 2.0 * w.bq * w.bk * w.d
+                                      / (s_attn * 1e-3) / 1e12, 2),
+            "what": "the same workload and step with theta = -1 (every block selective) and "
+                    "tau = 0.5: TopCdf drops blocks, Q K^T and P~V are skipped for them "
+                    "(Eq. 2); dense-equivalent TOPS over the step time; not the headline"}
 
     # ---- end to end through the public API with host buffers.  Every step
     # copies its inputs from pinned host memory and its output back, pipelined
@@ -396,8 +478,11 @@ def run_native(args, rank, world, local_rank):
     mma_flops = (qk_blocks + pv_blocks) * blk_flops
     achieved = mma_flops / (attn_ms * 1e-3) / 1e12
     peaks, peak_src = load_peaks()
-    peak = float(peaks["bf16_tflops_sustained"])
-    peak_burst = float(peaks["bf16_tflops"])
+    # the kernel runs back to back for seconds: the sustained (power-capped)
+    # peak applies; the burst figure is reported beside it
+    peak = attn_peak_tflops(w, peaks, qk_blocks, pv_blocks)
+    peak_burst = attn_peak_tflops(w, peaks, qk_blocks, pv_blocks, key="bf16_tflops")
+    peak_bf16 = float(peaks["bf16_tflops_sustained"])
     traffic = profiled_traffic(w.name, w.N)
     pbytes = pool_bytes(w)
     hbm_peak = float(peaks["hbm_gbs"])
@@ -414,14 +499,7 @@ def run_native(args, rank, world, local_rank):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int8-qk/f16-pv" if w.qk_int8 else ("bf16" if w.dtype == "bf16" else "f16"),
         "data": "synthetic (seeded generators; no model weights)",
-        "config": {"workload": f"{w.name}: B{w.B} Hq{w.Hq} Hkv{w.Hkv} N{w.N} d{w.d} "
-                               f"{w.dtype} causal={int(w.causal)} int8_qk={int(w.qk_int8)} "
-                               f"tau={w.tau} theta={w.theta} lambda={w.lam}",
-                   "global_batch": w.B * world, "seq_len": w.N,
-                   "parallelism": f"replicas x{world}",
-                   "l2": "inputs larger than L2 (no flush)" if _bytes(t) > L2_BYTES
-                   else "inputs fit in L2: 256 MB rewritten, then 256 MB read, between "
-                        "steps; steps timed alone"},
+        "config": workload_config(w, world, _bytes(t)),
         "latency_ms": {"predict": round(pred_ms, 4), "predict_pool": round(pool_ms, 4),
                        "predict_select": round(sel_ms, 4), "attention": round(attn_ms, 4),
                        "step": round(ms_step, 4), "step_median": round(step_median_ms, 4),
@@ -432,8 +510,11 @@ def run_native(args, rank, world, local_rank):
                      "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(pbytes / (pool_ms * 1e-3) / 1e9 / hbm_peak, 4),
                      "bytes_per_launch": pbytes,
-                     "kernel": "pool_kernel (+ k-bar and the K-code pass with INT8), "
-                               "algorithmic bytes / stage time"},
+                     "extra_bytes": pool_extra_bytes(w),
+                     "kernel": "pooling stage (pool_kernel; with INT8 also k-bar and the codes "
+                               "of K - k-bar): algorithmic bytes (one read of Q and K, means, "
+                               "self-similarities, codes, scales) / stage time; extra_bytes: "
+                               "the second read of K and the k-bar sums, not counted"},
             **({"permute": {"bound": "hbm", "unit": "GB/s", "peak": hbm_peak,
                             "bytes_per_launch": 2 * _bytes(t),
                             "achieved": round(2 * _bytes(t) / (perm_ms * 1e-3) / 1e9, 1),
@@ -459,27 +540,30 @@ def run_native(args, rank, world, local_rank):
         "sparsity": sparsity,
         "work": {"tiles": tiles, "qk_blocks": qk_blocks, "pv_blocks": pv_blocks,
                  "pv_slices": pv_slices, "skipped_slices": skipped, "visible_blocks": vis},
-        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": peak,
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(peak, 1),
                      "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
                      "traffic": traffic,
-                     "peak_source": f"{peak_src} bf16 sustained (MEASURED_PEAKS.json)",
+                     "peak_source": (f"{peak_src} sustained peaks (MEASURED_PEAKS.json) of each "
+                                     "contraction's dtype: "
+                                     + ("Q K^T INT8 at 2x the bf16 rate, " if w.qk_int8
+                                        else "Q K^T at the bf16 rate, ")
+                                     + "P~V fp16 at the bf16 rate; flop-weighted harmonic mean"),
                      "frac_of_burst_peak": round(achieved / peak_burst, 4),
+                     # Q K^T counted at the bf16 rate (as if it were a bf16 product)
+                     "frac_bf16_counted": round(achieved / peak_bf16, 4),
                      # NVIDIA's B200 datasheet: 2.25 PFLOP/s dense bf16 per GPU (the
                      # 4.5 figure printed beside it assumes 2:4 sparsity)
-                     "frac_of_datasheet_peak": round(achieved / DATASHEET_BF16_TFLOPS, 4),
-                     # INT8 Q K^T runs at twice the bf16 rate: the time the issued MMAs
-                     # need at the (sustained) peaks of their own dtypes, over the time taken
-                     "frac_mixed_peak": round(
-                         (qk_blocks * blk_flops / (2.0 if w.qk_int8 else 1.0)
-                          + pv_blocks * blk_flops) / (peak * 1e12) / (attn_ms * 1e-3), 4),
+                     "frac_of_datasheet_bf16": round(achieved / DATASHEET_BF16_TFLOPS, 4),
                      "kernel": "attn_kernel (tcgen05), issued MMA flops per launch / launch time"},
         "gpu_launches": launches_per_step * args.steps,
+        **({"sparse_regime": sparse} if sparse else {}),
         **({"graph": graph_line} if graph_line else {}),
         "clocks": clocks,
         "e2e": e2e,
     }
     if not args.no_cpu_baseline and world == 1:
-        line["cpu_baseline"] = cpu_baseline(w, t, tiles_per_sample=args.cpu_tiles)
+        line["cpu_baseline"], line["parity_sample"] = cpu_baseline(
+            w, t, tiles_per_sample=args.cpu_tiles, gpu_mask_h0=mask_h0)
     return line
 
 
@@ -520,10 +604,11 @@ def _visible_blocks(w):
 # CPU oracle on a bounded sample
 # ----------------------------------------------------------------------------
 
-def _oracle_sample(w, t, n_tiles, head=0):
+def _oracle_sample(w, t, n_tiles, head=0, details=False):
     """Oracle time for head `head`: the whole-sequence predictor prorated to
     n_tiles tiles, plus attention on n_tiles evenly spaced query tiles.
-    Returns (dense-equivalent ops of those tiles, seconds)."""
+    Returns (dense-equivalent ops of those tiles, seconds, tiles) and, with
+    details, the oracle's prediction and attention counters too."""
     from oracle import sparge_oracle as orc
     from synth import to_f64
     hk = head // (w.Hq // w.Hkv)
@@ -542,15 +627,16 @@ def _oracle_sample(w, t, n_tiles, head=0):
         if w.qk_int8 else None
     tiles = sorted({int(x) for x in np.linspace(0, Tm - 1, n_tiles)})
     t1 = time.perf_counter()
-    orc.sparse_attention(Q, K, V, idx, cnt, w.bq, w.bk, w.lam, w.causal, w.scale, quant=quant,
-                         tiles=[(0, 0, i) for i in tiles])
+    _, ost = orc.sparse_attention(Q, K, V, idx, cnt, w.bq, w.bk, w.lam, w.causal, w.scale,
+                                  quant=quant, tiles=[(0, 0, i) for i in tiles])
     t_attn = time.perf_counter() - t1
     pairs = 0
     for i in tiles:
         r0, r1 = i * w.bq, min(w.N, (i + 1) * w.bq)
         pairs += sum((r + 1) if w.causal else w.N for r in range(r0, r1))
     ops = 4.0 * w.d * pairs
-    return ops, t_attn + t_pred * len(tiles) / Tm, len(tiles)
+    out = (ops, t_attn + t_pred * len(tiles) / Tm, len(tiles))
+    return out + ((pr, ost),) if details else out
 
 
 def _blas_threads():
@@ -562,13 +648,27 @@ def _blas_threads():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(w, t, tiles_per_sample=64):
-    ops, sec, n = _oracle_sample(w, t, tiles_per_sample)
-    return {"value": round(ops / sec / 1e12, 9), "unit": "TOPS", "cores": _blas_threads(),
+def cpu_baseline(w, t, tiles_per_sample=64, gpu_mask_h0=None):
+    """The oracle timed on a bounded sample, and the parity counts that the
+    sample yields for head 0: the oracle's ambiguous mask entries, where the
+    GPU's mask differs from it, and the lambda decisions near the threshold
+    on the sampled tiles (the INT8 path's decisions use exact scores here)."""
+    ops, sec, n, (pr, ost) = _oracle_sample(w, t, tiles_per_sample, details=True)
+    base = {"value": round(ops / sec / 1e12, 9), "unit": "TOPS", "cores": _blas_threads(),
             "kind": "oracle",
             "sample": f"head 0: float64 oracle predictor over all {w.N} tokens (time prorated "
                       f"to the sample) + attention on {n} evenly spaced query tiles; "
                       f"{sec:.1f} s of CPU"}
+    vis = int(pr["visible"].sum()) * w.B
+    par = {"head": 0, "visible_blocks": vis, "kept_oracle": int(pr["M"].sum()),
+           "ambiguous_near_cut": int(pr["amb_cut"].sum()),
+           "ambiguous_near_theta": int(pr["amb_theta"].sum()),
+           "near_lambda_decisions": int(ost["near_lambda"]), "sampled_tiles": n}
+    if gpu_mask_h0 is not None:
+        diff = gpu_mask_h0 != pr["M"][:, 0]
+        par["mask_differing"] = int(diff.sum())
+        par["mask_differing_outside_ambiguous"] = int((diff & ~pr["amb"][:, 0]).sum())
+    return base, par
 
 
 def run_reference(args, rank, world):
@@ -590,12 +690,13 @@ def run_reference(args, rank, world):
               f"attention on {n_t} evenly spaced query tiles per step")
     return {"metric": METRIC, "value": round(value, 9), "unit": "TOPS", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(1e3 * dense_equiv_ops(w) / (value * 1e12), 1),
+            # the time each sampled step took; the whole workload would take
+            # ms_per_step_full_workload at the same rate
+            "ms_per_step": round(1e3 * tot_s / args.steps, 1),
+            "ms_per_step_full_workload": round(1e3 * dense_equiv_ops(w) / (value * 1e12), 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f64", "data": "synthetic (seeded generators; no model weights)",
-            "config": {"workload": f"{w.name}: B{w.B} Hq{w.Hq} Hkv{w.Hkv} N{w.N} d{w.d} "
-                                   f"{w.dtype} causal={int(w.causal)} int8_qk={int(w.qk_int8)}",
-                       "global_batch": w.B, "seq_len": w.N, "parallelism": "cpu"},
+            "config": workload_config(w, world, _bytes(t)),
             "impl": "reference",
             "cpu_baseline": {"value": round(value, 9), "unit": "TOPS", "cores": cores,
                              "kind": "oracle", "sample": sample},
@@ -752,6 +853,7 @@ def main():
     ap.add_argument("--graph", action="store_true",
                     help="also time the step captured into a CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sparse-regime", action="store_true")
     ap.add_argument("--cpu-tiles", type=int, default=64)
     ap.add_argument("--ref-tiles", type=int, default=4)
     ap.add_argument("--sweep", choices=("table6", "length", "tau", "permutation"), default=None,

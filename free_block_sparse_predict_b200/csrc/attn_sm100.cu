@@ -100,37 +100,6 @@ __device__ __forceinline__ void report_timeout(int32_t* status, volatile int* ab
   atomicExch(status, int32_t(SPARGE_ETIMEOUT));
 }
 
-// Whether a quarter of the exponentials run on the FMA pipe (exp2_poly2)
-// instead of the MUFU.  Off: once the INT8 scores stopped using the
-// conversion unit (which shares the MUFU pipe), all-MUFU measured 2-3% faster.
-constexpr bool kExp2OnFma = false;
-
-// 2^y for y <= 8 on the FMA pipe, for two values at once.  y = n + f with
-// n = round(y) (adding and subtracting 1.5 * 2^23) and f in [-1/2, 1/2];
-// 2^f by the cubic p(f) that minimises the maximum relative error on that
-// interval (Remez exchange; coefficients from exp2_poly.py, relative error
-// 7.5e-5); 2^n by adding n to the exponent field.  y is clamped at -125 so the
-// exponent never leaves the normal range (2^-125 is 0 for every later use).
-__device__ __forceinline__ void exp2_poly2(float y0, float y1, float& r0, float& r1) {
-  constexpr float kC0 = 9.999280572e-01f, kC1 = 6.932609677e-01f;
-  constexpr float kC2 = 2.426111251e-01f, kC3 = 5.517166853e-02f;
-  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-  y0 = fmaxf(y0, -125.f);
-  y1 = fmaxf(y1, -125.f);
-  const uint64_t y = pack2(y0, y1);
-  const uint64_t t = add2(y, pack2(kMagic, kMagic));
-  const uint64_t nn = add2(t, pack2(-kMagic, -kMagic));
-  const uint64_t f = fma2(nn, pack2(-1.f, -1.f), y);
-  uint64_t p = fma2(pack2(kC3, kC3), f, pack2(kC2, kC2));
-  p = fma2(p, f, pack2(kC1, kC1));
-  p = fma2(p, f, pack2(kC0, kC0));
-  float p0, p1, t0, t1;
-  unpack2(p, p0, p1);
-  unpack2(t, t0, t1);
-  r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-  r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-}
-
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -427,7 +396,6 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const __grid_constant
       }
       if (grow) m_sc = m_new;
       // P~ = 2^(x * sc - m_sc): one packed FMA per pair, then ex2 on the MUFU
-      // (with kExp2OnFma, the FMA-pipe polynomial for one pair in four)
       const float nb = (m_sc == -INFINITY) ? 0.f : -m_sc;
       const uint64_t sc2 = pack2(sc, sc), nb2 = pack2(nb, nb);
       float pv[64];
@@ -437,12 +405,8 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const __grid_constant
         if (MODE == kI8) x2 = add2(x2, pack2(-kMagic, -kMagic));  // exact
         float y0, y1;
         unpack2(fma2(x2, sc2, nb2), y0, y1);
-        if (kExp2OnFma && (c & 7) == 6) {
-          exp2_poly2(y0, y1, pv[c], pv[c + 1]);
-        } else {
-          pv[c] = ex2_approx(y0);
-          pv[c + 1] = ex2_approx(y1);
-        }
+        pv[c] = ex2_approx(y0);
+        pv[c + 1] = ex2_approx(y1);
       }
       if (lim < 64) {
 #pragma unroll

@@ -7,11 +7,11 @@
 //
 // The array is a fixed kNoAllocScratchBytes (32 MiB) per GPU; every GPU that
 // loads the library holds it until the process exits.  All calls share it and
-// it keeps the last call's contents: the status word of the kernels' bounded
-// waits is cleared at the start of every call, every other region is
-// completely rewritten by the pooling kernel before any kernel reads it, and
-// two calls whose kernels overlap on the GPU (different streams, no ordering
-// between them) race on it.
+// it keeps the last call's contents: every region is completely rewritten by
+// the pooling kernel before any kernel reads it, so nothing has to be cleared,
+// and two calls whose kernels overlap on the GPU (different streams, no
+// ordering between them) race on it.  The predictor's kernels have no
+// device-side waits, so there is no status word to report.
 #include <cstdint>
 #include <mutex>
 
@@ -53,7 +53,9 @@ extern "C" sparge_status_t sparge_predict_mask_noalloc(const sparge_params_t* p,
                                                        int32_t* kv_idx, int32_t* kv_cnt,
                                                        float* s_q, float* s_k,
                                                        cudaStream_t stream) {
-  if (p == nullptr || sparge_workspace_bytes(p) == 0) return SPARGE_EINVAL;
+  // the same parameter check, and so the same status codes, as sparge_predict_mask
+  sparge_status_t st = check_params(p);
+  if (st != SPARGE_OK) return st;
   if (p->qk_int8) return SPARGE_EUNSUPPORTED;  // the INT8 codes must outlive the call
   if (p->B == 0 || p->N == 0) return SPARGE_OK;
   if (q == nullptr || k == nullptr || mask == nullptr || kv_idx == nullptr || kv_cnt == nullptr)
@@ -68,18 +70,10 @@ extern "C" sparge_status_t sparge_predict_mask_noalloc(const sparge_params_t* p,
   if (L.s_k + align256(size_t(p->B) * p->Hkv * cdiv(p->N, p->bk) * 4) > kNoAllocScratchBytes)
     return SPARGE_EWORKSPACE;
 
-  cudaPointerAttributes attr;
-  if (cudaPointerGetAttributes(&attr, q) != cudaSuccess) {
-    cudaGetLastError();
-    return SPARGE_EINVAL;
-  }
-  if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged)
-    return SPARGE_EINVAL;
-  int cur = -1;
-  if (cudaGetDevice(&cur) != cudaSuccess) return SPARGE_ECUDA;
-  if (cur != attr.device && cudaSetDevice(attr.device) != cudaSuccess) return SPARGE_ECUDA;
+  DeviceScope dev;
+  if ((st = dev.enter(q)) != SPARGE_OK) return st;
   void* scratch = nullptr;
-  if (scratch_address(attr.device, &scratch) != cudaSuccess) return SPARGE_ECUDA;
+  if (scratch_address(dev.device(), &scratch) != cudaSuccess) return SPARGE_ECUDA;
 
   PredictPtrs x{};
   x.q = q;
@@ -91,9 +85,7 @@ extern "C" sparge_status_t sparge_predict_mask_noalloc(const sparge_params_t* p,
   x.mask = mask;
   x.kv_idx = kv_idx;
   x.kv_cnt = kv_cnt;
-  // the status word of the kernels' bounded waits must start at zero
-  x.status = ws_ptr<int32_t>(scratch, L.status);
-  if (cudaMemsetAsync(x.status, 0, sizeof(int32_t), stream) != cudaSuccess) return SPARGE_ECUDA;
+  x.status = nullptr;  // the predictor's kernels have no device-side waits to report
   if (launch_predict(*p, x, stream) != cudaSuccess) return SPARGE_ECUDA;
   const int64_t Tm = cdiv(p->N, p->bq), Tn = cdiv(p->N, p->bk);
   if (s_q != nullptr && cudaMemcpyAsync(s_q, x.s_q, size_t(p->B) * p->Hq * Tm * 4,

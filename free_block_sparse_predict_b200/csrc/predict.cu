@@ -6,7 +6,9 @@
 //                   CosSim (Eq. 6, read as the mean of the block's token cosine
 //                   matrix), via mean_{a,b} xh_a.xh_b = |sum_a xh_a|^2 / n^2.
 //                   With INT8 it also quantises Q per block (Algorithm 1 step 2).
-//   kbar_*_kernel   per-head mean of K from the block means (K smoothing).
+//   pool_kernel<.., 2>  with INT8, the pooling pass over K alone, which also
+//                   writes each K block's float64 column sums;
+//   kbar_*_kernel   per-head mean of K from them (K smoothing);
 //   pool_kernel<.., 1>  per-block INT8 of K - kbar (second pass over K).
 //   select_kernel   per query block: S_hat = scale q_i k^T with -inf columns
 //                   (Eq. 7), row softmax, TopCdf(tau) (Eq. 8) by an exact
@@ -45,6 +47,7 @@ struct PoolArgs {
   const float* kbar; // INT8 pass over K - kbar
   int8_t* k_codes;
   float* dk;
+  double* ksum64;    // KIND 2: [B, Hkv, Tn, D] float64 column sums of the K blocks
   int32_t* status;
 };
 
@@ -62,6 +65,12 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
 __device__ __forceinline__ uint4 opaque(uint4 v) {
   asm volatile("" : "+r"(v.x), "+r"(v.y), "+r"(v.z), "+r"(v.w));
   return v;
+}
+
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
 }
 
 __device__ __forceinline__ void named_barrier(int id, int threads) {
@@ -96,29 +105,78 @@ __device__ __forceinline__ float absmax2_value(uint32_t acc) {
   return fmaxf(f.x, f.y);
 }
 
-// Eight INT8 codes rint(x * inv) of a packed fp32 row chunk.  q = x * inv is
-// the IEEE-rounded fp32 product (__fmul_rn), then q + 1.5 * 2^23 (__fadd_rn)
-// rounds q to the nearest integer, ties to even, exactly as rint does for
-// |q| < 2^22; |q| <= 127 (x is bounded by the absmax that inv comes from), so
-// the code is the low byte of that sum's bits, two's complement included.
-// Scalar on purpose: with the packed f32x2 forms the compiler fused the
-// product into the add, rounding the exact product instead of q, which turns
-// ties such as q = 63.5 (from a product just below it) the other way.
-__device__ __forceinline__ uint2 codes8(const uint64_t (&x2)[4], float inv) {
+// rint(x / delta) of eight values by the IEEE division itself, as the bits
+// of q + 1.5 * 2^23 (the code is their low byte).  Out of line: it runs for
+// about one call in a thousand, and inlined into every unrolled row of the
+// pooling kernel it made the kernel's code too large to stay in the
+// instruction cache.
+__device__ __noinline__ uint2 codes8_exact(float x0, float x1, float x2, float x3, float x4,
+                                           float x5, float x6, float x7, float delta) {
   constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  const float x[8] = {x0, x1, x2, x3, x4, x5, x6, x7};
   uint32_t bits[8];
 #pragma unroll
+  for (int i = 0; i < 8; ++i) bits[i] = __float_as_uint(__fadd_rn(__fdiv_rn(x[i], delta), kMagic));
+  const uint32_t lo = __byte_perm(__byte_perm(bits[0], bits[1], 0x0040),
+                                  __byte_perm(bits[2], bits[3], 0x0040), 0x5410);
+  const uint32_t hi = __byte_perm(__byte_perm(bits[4], bits[5], 0x0040),
+                                  __byte_perm(bits[6], bits[7], 0x0040), 0x5410);
+  return make_uint2(lo, hi);
+}
+
+// Eight INT8 codes rint(x / delta): round half to even of the IEEE float32
+// quotient.  Fast path: t = x * inv with inv = 1/delta correctly rounded,
+// then t + 1.5 * 2^23 rounds t to the nearest integer, ties to even, exactly
+// (|t| < 2^22), and the code is the low byte of that sum's bits, two's
+// complement included.  t differs from the quotient fl(x / delta) by less than
+// 1.9e-5 (|x / delta| <= 127.00001, two roundings of 2^-24 relative each, and
+// the quotient's own half ulp of 2^-18), so rint(t) is rint(fl(x / delta))
+// unless t lies within 2^-14 of a half-integer.  Those take the slow path:
+// the IEEE division itself.  The products and sums are explicit .rn
+// instructions, so none is fused.
+__device__ __forceinline__ uint2 codes8(const uint64_t (&x2)[4], float inv, float delta,
+                                        bool exact_only) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  constexpr float kNear = 0.5f - 1.0f / 16384.0f;
+  const uint64_t inv2 = pack2(inv, inv), mg2 = pack2(kMagic, kMagic);
+  uint32_t bits[8];
+  float dmax = 0.f;
+#pragma unroll
   for (int i = 0; i < 4; ++i) {
-    float a, b;
-    unpack2(x2[i], a, b);
-    bits[2 * i] = __float_as_uint(__fadd_rn(__fmul_rn(a, inv), kMagic));
-    bits[2 * i + 1] = __float_as_uint(__fadd_rn(__fmul_rn(b, inv), kMagic));
+    const uint64_t t2 = mul2(x2[i], inv2);
+    const uint64_t r2 = add2(t2, mg2);
+    const uint64_t d2 = sub2(t2, sub2(r2, mg2));  // t - rint(t), exact
+    float r0, r1, d0, d1;
+    unpack2(r2, r0, r1);
+    unpack2(d2, d0, d1);
+    bits[2 * i] = __float_as_uint(r0);
+    bits[2 * i + 1] = __float_as_uint(r1);
+    dmax = fmax3(dmax, fabsf(d0), fabsf(d1));
+  }
+  // (a NaN distance fails the test and also takes the exact path)
+  if (exact_only || !(dmax <= kNear)) {
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) unpack2(x2[i], v[2 * i], v[2 * i + 1]);
+    return codes8_exact(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7], delta);
   }
   const uint32_t lo = __byte_perm(__byte_perm(bits[0], bits[1], 0x0040),
                                   __byte_perm(bits[2], bits[3], 0x0040), 0x5410);
   const uint32_t hi = __byte_perm(__byte_perm(bits[4], bits[5], 0x0040),
                                   __byte_perm(bits[6], bits[7], 0x0040), 0x5410);
   return make_uint2(lo, hi);
+}
+
+// A float32 value as float64, built from its bits (the fp64 conversion unit
+// runs at a quarter of the integer rate): exponent rebiased by 1023 - 127,
+// significand moved down three places into the high word.  Exact for every
+// float32 whose low three significand bits are zero, which holds for every
+// widened bf16 or f16 value; zeros stay zero and float32 subnormals (only a
+// bf16 below 2^-126 widens to one) are flushed to zero.
+__device__ __forceinline__ double f32_to_f64_bits(float x) {
+  const uint32_t f = __float_as_uint(x), m = f & 0x7FFFFFFFu;
+  const uint32_t hi = (f & 0x80000000u) | (m >= 0x00800000u ? (m >> 3) + 0x38000000u : 0u);
+  return __hiloint2double(int(hi), 0);
 }
 
 // One warp per SLAB-row slab of a block, held in registers for the whole
@@ -135,9 +193,15 @@ __device__ __forceinline__ uint2 codes8(const uint64_t (&x2)[4], float inv) {
 // does not depend on scheduling.
 //   KIND 0  pooling pass over Q blocks then K blocks: mean token, CosSim by
 //           |sum xhat|^2 / n^2, and with q_codes the INT8 codes of Q.
-//   KIND 1  INT8 pass over K blocks: codes of K - kbar and their scales.
+//   KIND 1  INT8 pass over K blocks, last block first (the blocks pooled last
+//           are still in L2): codes of K - kbar and their scales.
+//   KIND 2  pooling pass over K blocks that also writes every block's column
+//           sums in float64 (exact for 16-bit inputs), from which kbar is the
+//           float64 mean rounded once to float32.
 template <int D, bool BF16, int KIND, int SLAB>
 __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(PoolArgs a) {
+  constexpr bool POOL = KIND != 1;
+  constexpr bool SUM64 = KIND == 2;
   constexpr int CH = D * 2 / 16;  // lanes per row
   constexpr int RPW = 32 / CH;    // rows per warp-wide load
   constexpr int NR = SLAB / RPW;  // rows per lane
@@ -148,6 +212,7 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
   static_assert(NR % CH == 0, "butterfly needs NR a multiple of CH");
   __shared__ float part[WARPS][2 * D];
   __shared__ float pmax[WARPS];
+  __shared__ double part64[SUM64 ? WARPS : 1][SUM64 ? D : 1];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t gw = int64_t(blockIdx.x) * WARPS + warp;
@@ -155,9 +220,11 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
   const bool isQ = KIND == 0 && gw < nQw;
   const int G = isQ ? GQ : GK;
   const int64_t rel = isQ ? gw : gw - nQw;
-  const int64_t blkid = rel / G;
+  const int64_t nb = isQ ? a.nQblocks : a.nblocks - a.nQblocks;
+  int64_t blkid = rel / G;
   const int sub = int(rel % G);  // slab index inside the block
-  if (blkid >= (isQ ? a.nQblocks : a.nblocks - a.nQblocks)) return;  // whole groups leave
+  if (blkid >= nb) return;  // whole groups leave
+  if (KIND == 1) blkid = nb - 1 - blkid;
   const int T = isQ ? a.Tm : a.Tn;
   const int BLK = isQ ? kPoolBQ : kPoolBK;
   const int64_t bh = blkid / T;
@@ -188,7 +255,10 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
   float inv_own[R];
   const int group_base = lane & ~(CH - 1);
   const int w0 = warp - sub;
-  if (KIND == 0) {
+  double s64[SUM64 ? 8 : 1];  // float64 column sums (KIND 2)
+#pragma unroll
+  for (int e = 0; e < (SUM64 ? 8 : 1); ++e) s64[e] = 0.0;
+  if (POOL) {
     // ---- pass 1: squared row norms (one value per row), column sums of x,
     // and the exact |x| max on the raw 16-bit halves
     float v[NR];
@@ -230,6 +300,22 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
     // lane c of a row group now holds rows c * R .. c * R + R - 1
 #pragma unroll
     for (int t = 0; t < R; ++t) inv_own[t] = v[t] > 0.f ? rsqrtf(v[t]) : 0.f;
+    if (SUM64) {
+      // a sweep of its own, once the row norms no longer hold registers;
+      // rows past the block are zero and add nothing
+#pragma unroll
+      for (int u = 0; u < NR; ++u) {
+        const uint4 rw = opaque(raw[u]);
+        const uint32_t w[4] = {rw.x, rw.y, rw.z, rw.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float x0, x1;
+          unpack2(widen2<BF16>(w[e]), x0, x1);
+          s64[2 * e] += f32_to_f64_bits(x0);
+          s64[2 * e + 1] += f32_to_f64_bits(x1);
+        }
+      }
+    }
   } else {
 #pragma unroll
     for (int u = 0; u < NR; ++u) {
@@ -246,33 +332,60 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  if (KIND == 0) {
+  if (POOL) {
 #pragma unroll
     for (int o = CH; o < 32; o <<= 1)
 #pragma unroll
       for (int e = 0; e < 8; ++e) sx[e] += __shfl_xor_sync(0xffffffffu, sx[e], o);
   }
+  if (SUM64) {
+#pragma unroll
+    for (int o = CH; o < 32; o <<= 1)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s64[e] += __shfl_xor_sync(0xffffffffu, s64[e], o);
+  }
   // ---- the block's absmax and column sums over its G slabs (slab order)
   if (G > 1) {
-    if (KIND == 0 && ro == 0) {
+    if (POOL && ro == 0) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) part[warp][c * 8 + e] = sx[e];
     }
+    if (SUM64 && ro == 0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) part64[warp][c * 8 + e] = s64[e];
+    }
     if (lane == 0) pmax[warp] = amax;
     named_barrier(1 + warp / G, 32 * G);
-    if (KIND == 0) {
+    if (POOL) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) sx[e] = part[w0][c * 8 + e];
       for (int g = 1; g < G; ++g)
 #pragma unroll
         for (int e = 0; e < 8; ++e) sx[e] += part[w0 + g][c * 8 + e];
     }
+    if (SUM64 && sub == 0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s64[e] = part64[w0][c * 8 + e];
+      for (int g = 1; g < G; ++g)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s64[e] += part64[w0 + g][c * 8 + e];
+    }
     amax = pmax[w0];
     for (int g = 1; g < G; ++g) amax = fmaxf(amax, pmax[w0 + g]);
   }
+  if (SUM64 && sub == 0 && ro == 0) {
+    double* dst = a.ksum64 + (bh * T + blk) * D + c * 8;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) dst[e] = s64[e];
+  }
   const bool quantise = KIND == 1 || (isQ && a.q_codes != nullptr);
-  const float inv = amax > 0.f ? 127.0f / amax : 0.f;
-  if (quantise && sub == 0 && lane == 0) (KIND == 1 ? a.dk : a.dq)[bh * T + blk] = amax / 127.0f;
+  // delta = absmax / 127 (IEEE divide); inv = 1 / delta correctly rounded.  A
+  // subnormal delta, whose reciprocal overflows, sends every code to the
+  // exact path.
+  const float delta = amax / 127.0f;
+  const float inv = delta > 0.f ? __frcp_rn(delta) : 0.f;
+  const bool exact_only = delta > 0.f && !(inv <= FLT_MAX);
+  if (quantise && sub == 0 && lane == 0) (KIND == 1 ? a.dk : a.dq)[bh * T + blk] = delta;
   int8_t* codes = quantise ? (KIND == 1 ? a.k_codes : a.q_codes) + row0 * D + c * 8 : nullptr;
   // ---- pass 2: column sums of x / |x_row| (and the codes, once absmax is known)
   uint64_t su2[4];
@@ -286,7 +399,7 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
     uint64_t x2[4];
 #pragma unroll
     for (int e = 0; e < 4; ++e) x2[e] = widen2<BF16>(w[e]);
-    if (KIND == 0) {
+    if (POOL) {
       const float iv = __shfl_sync(0xffffffffu, inv_own[u % R], group_base | (u / R));
       const uint64_t iv2 = pack2(iv, iv);
 #pragma unroll
@@ -295,9 +408,10 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
 #pragma unroll
       for (int e = 0; e < 4; ++e) x2[e] = add2(x2[e], nkb2[e]);
     }
-    if (quantise && r < srows) *reinterpret_cast<uint2*>(codes + int64_t(r) * D) = codes8(x2, inv);
+    if (quantise && r < srows)
+      *reinterpret_cast<uint2*>(codes + int64_t(r) * D) = codes8(x2, inv, delta, exact_only);
   }
-  if constexpr (KIND == 0) {
+  if constexpr (POOL) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) unpack2(su2[e], su[2 * e], su[2 * e + 1]);
 #pragma unroll
@@ -334,32 +448,33 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
   }
 }
 
-// kbar[bh, :] = (sum_j n_j * k_mean[bh, j, :]) / N in a fixed order: slice s
-// of kKbarSlices sums its key blocks into part[bh, s, :], then one CTA per head
-// adds the slices in index order.
+// kbar[bh, :] = fl32((sum over the N tokens of K[bh, :, :]) / N) with the sum
+// in float64, in a fixed order: slice s of kKbarSlices adds its key blocks'
+// float64 column sums into part[bh, s, :], then one CTA per head adds the
+// slices in index order.  For 16-bit K every partial sum is exact (the
+// exponents of realistic data span far fewer than 53 bits), so the result is
+// the float64 mean rounded once to float32, whatever the order.
 template <int D>
-__global__ void __launch_bounds__(D) kbar_partial_kernel(const float* k_mean, float* part,
-                                                         int32_t N, int32_t bk, int32_t Tn) {
+__global__ void __launch_bounds__(D) kbar_partial_kernel(const double* ksum, double* part,
+                                                         int32_t Tn) {
   const int64_t bh = blockIdx.x / kKbarSlices;
   const int sl = int(blockIdx.x % kKbarSlices), col = threadIdx.x;
   const int per = (Tn + kKbarSlices - 1) / kKbarSlices;
   const int j0 = sl * per, j1 = min(Tn, j0 + per);
-  float acc = 0.f;
-  for (int j = j0; j < j1; ++j) {
-    const int n = min(bk, N - j * bk);
-    acc = fmaf(k_mean[(bh * Tn + j) * D + col], float(n), acc);
-  }
+  double acc = 0.0;
+  for (int j = j0; j < j1; ++j) acc += ksum[(bh * Tn + j) * D + col];
   part[(bh * kKbarSlices + sl) * D + col] = acc;
 }
 
 template <int D>
-__global__ void __launch_bounds__(D) kbar_final_kernel(const float* part, float* kbar, int32_t N) {
+__global__ void __launch_bounds__(D) kbar_final_kernel(const double* part, float* kbar,
+                                                       int32_t N) {
   const int64_t bh = blockIdx.x;
   const int col = threadIdx.x;
-  float s = 0.f;
+  double s = 0.0;
 #pragma unroll 8
   for (int sl = 0; sl < kKbarSlices; ++sl) s += part[(bh * kKbarSlices + sl) * D + col];
-  kbar[bh * D + col] = s / float(N);
+  kbar[bh * D + col] = __double2float_rn(s / double(N));
 }
 
 // ------------------------------------------------------------------ select
@@ -391,6 +506,19 @@ __device__ __forceinline__ int visible_cols(int i, int N, int bq, int bk, int Tn
   return min(Tn, last_row / bk + 1);
 }
 
+// A fix row (Eq. 9): every visible block of query block i is kept, in order.
+// One warp.
+__device__ __forceinline__ void write_full_row(const SelectArgs& a, int64_t bh, int i) {
+  const int lane = threadIdx.x & 31;
+  const int nvis = visible_cols(i, a.N, a.bq, a.bk, a.Tn, a.causal);
+  const int64_t out = (bh * a.Tm + i) * a.Tn;
+  for (int j = lane; j < a.Tn; j += 32) {
+    a.mask[out + j] = j < nvis ? 1 : 0;
+    if (j < nvis) a.kv_idx[out + j] = j;
+  }
+  if (lane == 0) a.kv_cnt[bh * a.Tm + i] = nvis;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
   extern __shared__ __align__(16) float smem[];
@@ -405,6 +533,17 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
   const int tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
   const int i_last = min(a.Tm, i0 + kSelRows) - 1;
   const int jcount = visible_cols(i_last, a.N, a.bq, a.bk, a.Tn, a.causal);
+
+  // Eq. 9: a query block with s_q < theta is a fix block, its whole visible
+  // row is 1 and its S_hat, softmax and TopCdf decide nothing.  When every
+  // query block of this CTA is one, the S_hat phase is skipped.
+  const bool my_fix = tid >= kSelRows || i0 + tid >= a.Tm ||
+                      a.s_q[bh * a.Tm + i0 + tid] < a.theta;
+  if (__syncthreads_and(my_fix)) {
+    const int i = i0 + w;
+    if (i < a.Tm) write_full_row(a, bh, i);
+    return;
+  }
 
   for (int idx = tid; idx < kSelRows * D; idx += kSelThreads) {
     const int r = idx / D, e = idx % D;
@@ -473,6 +612,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
   float* row = shat + w * a.Tn;
   const int nvis = visible_cols(i, a.N, a.bq, a.bk, a.Tn, a.causal);
   const bool fix_row = a.s_q[bh * a.Tm + i] < a.theta;
+  if (fix_row) {
+    write_full_row(a, bh, i);
+    return;
+  }
   const float* sk = a.s_k + kbh * a.Tn;
 
   float mx = -INFINITY;
@@ -563,7 +706,7 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
     bool keep = false;
     if (j < nvis) {
       const float e = row[j];
-      keep = (e >= 0.f && e >= t_star) || fix_row || sk[j] < a.theta;
+      keep = (e >= 0.f && e >= t_star) || sk[j] < a.theta;
     }
     if (j < a.Tn) a.mask[out + j] = keep ? 1 : 0;
     const uint32_t bal = __ballot_sync(0xffffffffu, keep);
@@ -615,27 +758,42 @@ cudaError_t pool_impl(const sparge_params_t& p, const PredictPtrs& x, cudaStream
   cudaError_t e;
   constexpr int SLAB = D == 128 ? 32 : 64;  // 8 KB of bf16/f16 per warp
   constexpr int64_t warps_per_cta = kPoolThreads / 32;
-  const int64_t w0 = pa.nQblocks * (kPoolBQ / SLAB) + nK * (kPoolBK / SLAB);
-  pool_kernel<D, BF16, 0, SLAB><<<unsigned(cdiv(w0, warps_per_cta)), kPoolThreads, 0, s>>>(pa);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (x.k_codes != nullptr) {
-    const unsigned BHk = unsigned(int64_t(p.B) * p.Hkv);
-    kbar_partial_kernel<D><<<BHk * kKbarSlices, D, 0, s>>>(x.k_mean, x.kbar_part, p.N, p.bk,
-                                                            int32_t(Tn));
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    kbar_final_kernel<D><<<BHk, D, 0, s>>>(x.kbar_part, x.kbar, p.N);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    PoolArgs qa = pa;
-    qa.nblocks = nK;
-    qa.nQblocks = 0;
-    qa.kbar = x.kbar;
-    qa.k_codes = x.k_codes;
-    qa.dk = x.dk;
-    const int64_t w1 = nK * (kPoolBK / SLAB);
-    pool_kernel<D, BF16, 1, SLAB><<<unsigned(cdiv(w1, warps_per_cta)), kPoolThreads, 0, s>>>(qa);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  constexpr int64_t GQ = kPoolBQ / SLAB, GK = kPoolBK / SLAB;
+  if (x.k_codes == nullptr) {
+    // one pass over Q then K blocks
+    const int64_t w0 = pa.nQblocks * GQ + nK * GK;
+    pool_kernel<D, BF16, 0, SLAB><<<unsigned(cdiv(w0, warps_per_cta)), kPoolThreads, 0, s>>>(pa);
+    return cudaGetLastError();
   }
-  return cudaSuccess;
+  if constexpr (D != 128) {
+    return cudaErrorInvalidValue;  // the INT8 path exists for d = 128 only
+  } else {
+  // INT8: K first -- pooling with float64 column sums, kbar, then the codes of
+  // K - kbar (last blocks first, while they are still in L2) -- then Q's
+  // pooling pass, which also writes the Q codes.
+  PoolArgs ka = pa;
+  ka.nQblocks = 0;
+  ka.nblocks = nK;
+  ka.ksum64 = x.ksum64;
+  pool_kernel<D, BF16, 2, SLAB><<<unsigned(cdiv(nK * GK, warps_per_cta)), kPoolThreads, 0, s>>>(ka);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const unsigned BHk = unsigned(int64_t(p.B) * p.Hkv);
+  kbar_partial_kernel<D><<<BHk * kKbarSlices, D, 0, s>>>(x.ksum64, x.kbar_part, int32_t(Tn));
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  kbar_final_kernel<D><<<BHk, D, 0, s>>>(x.kbar_part, x.kbar, p.N);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  PoolArgs ca = ka;
+  ca.kbar = x.kbar;
+  ca.k_codes = x.k_codes;
+  ca.dk = x.dk;
+  pool_kernel<D, BF16, 1, SLAB><<<unsigned(cdiv(nK * GK, warps_per_cta)), kPoolThreads, 0, s>>>(ca);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  PoolArgs qa = pa;
+  qa.nblocks = qa.nQblocks;
+  pool_kernel<D, BF16, 0, SLAB>
+      <<<unsigned(cdiv(qa.nQblocks * GQ, warps_per_cta)), kPoolThreads, 0, s>>>(qa);
+  return cudaGetLastError();
+  }
 }
 
 template <int D>

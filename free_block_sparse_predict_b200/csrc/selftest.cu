@@ -33,15 +33,9 @@ using namespace sparge;
 
 extern "C" sparge_status_t sparge_selftest_wait_timeout(void* ws, cudaStream_t stream) {
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SPARGE_EINVAL;
-  cudaPointerAttributes a;
-  if (cudaPointerGetAttributes(&a, ws) != cudaSuccess) {
-    cudaGetLastError();
-    return SPARGE_EINVAL;
-  }
-  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return SPARGE_EINVAL;
-  int cur = -1;
-  if (cudaGetDevice(&cur) != cudaSuccess) return SPARGE_ECUDA;
-  if (cur != a.device && cudaSetDevice(a.device) != cudaSuccess) return SPARGE_ECUDA;
+  DeviceScope dev;
+  const sparge_status_t st = dev.enter(ws);
+  if (st != SPARGE_OK) return st;
   unsatisfiable_wait_kernel<<<1, 32, 0, stream>>>(static_cast<int32_t*>(ws));
   return cudaGetLastError() == cudaSuccess ? SPARGE_OK : SPARGE_ECUDA;
 }

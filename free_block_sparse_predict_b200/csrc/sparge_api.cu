@@ -15,6 +15,20 @@ constexpr int64_t kMaxTn = 5952;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+bool empty_problem(const sparge_params_t* p) { return p->B == 0 || p->N == 0; }
+
+sparge_status_t from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return SPARGE_OK;
+  if (e == cudaErrorNotSupported) return SPARGE_EUNSUPPORTED;
+  return SPARGE_ECUDA;
+}
+
+int elem_size(sparge_dtype_t t) { return t == SPARGE_F32 ? 4 : 2; }
+
+}  // namespace
+
+namespace sparge {
+
 sparge_status_t check_params(const sparge_params_t* p) {
   if (p == nullptr) return SPARGE_EINVAL;
   if (p->B < 0 || p->N < 0 || p->Hq < 1 || p->Hkv < 1 || p->d < 1) return SPARGE_EINVAL;
@@ -36,31 +50,7 @@ sparge_status_t check_params(const sparge_params_t* p) {
   return SPARGE_OK;
 }
 
-bool empty_problem(const sparge_params_t* p) { return p->B == 0 || p->N == 0; }
-
-// Make the library's runtime target the device that owns ptr.
-sparge_status_t select_device(const void* ptr) {
-  cudaPointerAttributes a;
-  if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
-    cudaGetLastError();
-    return SPARGE_EINVAL;
-  }
-  if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return SPARGE_EINVAL;
-  int cur = -1;
-  if (cudaGetDevice(&cur) != cudaSuccess) return SPARGE_ECUDA;
-  if (cur != a.device && cudaSetDevice(a.device) != cudaSuccess) return SPARGE_ECUDA;
-  return SPARGE_OK;
-}
-
-sparge_status_t from_cuda(cudaError_t e) {
-  if (e == cudaSuccess) return SPARGE_OK;
-  if (e == cudaErrorNotSupported) return SPARGE_EUNSUPPORTED;
-  return SPARGE_ECUDA;
-}
-
-int elem_size(sparge_dtype_t t) { return t == SPARGE_F32 ? 4 : 2; }
-
-}  // namespace
+}  // namespace sparge
 
 extern "C" {
 
@@ -83,7 +73,8 @@ sparge_status_t sparge_hilbert_index(int32_t N, int32_t prefix_len, int32_t T, i
   if (N == 0) return SPARGE_OK;
   if (perm == nullptr || ws == nullptr || (reinterpret_cast<uintptr_t>(perm) & 3u)) return SPARGE_EINVAL;
   if (ws_bytes < need) return SPARGE_EWORKSPACE;
-  sparge_status_t st = select_device(perm);
+  DeviceScope dev;
+  sparge_status_t st = dev.enter(perm);
   if (st != SPARGE_OK) return st;
   return from_cuda(launch_hilbert_index(N, prefix_len, T, Hg, Wg, perm, ws, stream));
 }
@@ -103,7 +94,8 @@ static sparge_status_t permute_common(const void* src, void* dst, int32_t B, int
   const char* s0 = static_cast<const char*>(src);
   const char* d0 = static_cast<const char*>(dst);
   if (s0 < d0 + bytes && d0 < s0 + bytes) return SPARGE_EINVAL;  // overlap
-  sparge_status_t st = select_device(dst);
+  DeviceScope dev;
+  sparge_status_t st = dev.enter(dst);
   if (st != SPARGE_OK) return st;
   return from_cuda(
       launch_permute_rows(src, dst, int64_t(B) * H, N, int32_t(row_bytes), perm, inverse, stream));
@@ -144,7 +136,8 @@ static sparge_status_t predict_common(int stages, const sparge_params_t* p, cons
   }
   const WsLayout L = ws_layout(*p);
   if (ws_bytes < L.total) return SPARGE_EWORKSPACE;
-  if ((st = select_device((stages & kStagePool) ? q : ws)) != SPARGE_OK) return st;
+  DeviceScope dev;
+  if ((st = dev.enter((stages & kStagePool) ? q : ws)) != SPARGE_OK) return st;
   PredictPtrs x{};
   x.q = q;
   x.k = k;
@@ -158,7 +151,8 @@ static sparge_status_t predict_common(int stages, const sparge_params_t* p, cons
     x.dq = ws_ptr<float>(ws, L.dq);
     x.dk = ws_ptr<float>(ws, L.dk);
     x.kbar = ws_ptr<float>(ws, L.kbar);
-    x.kbar_part = ws_ptr<float>(ws, L.kbar_part);
+    x.kbar_part = ws_ptr<double>(ws, L.kbar_part);
+    x.ksum64 = ws_ptr<double>(ws, L.k_sum64);
   }
   x.mask = mask;
   x.kv_idx = kv_idx;
@@ -211,7 +205,8 @@ sparge_status_t sparge_mask_compact(const sparge_params_t* p, const uint8_t* mas
   if (mask == nullptr || kv_idx == nullptr || kv_cnt == nullptr) return SPARGE_EINVAL;
   if ((reinterpret_cast<uintptr_t>(kv_idx) & 3u) || (reinterpret_cast<uintptr_t>(kv_cnt) & 3u))
     return SPARGE_EINVAL;
-  if ((st = select_device(kv_idx)) != SPARGE_OK) return st;
+  DeviceScope dev;
+  if ((st = dev.enter(kv_idx)) != SPARGE_OK) return st;
   return from_cuda(launch_mask_compact(*p, mask, kv_idx, kv_cnt, stream));
 }
 
@@ -231,7 +226,8 @@ sparge_status_t sparge_attn_fwd(const sparge_params_t* p, const void* q, const v
     return SPARGE_EINVAL;
   const WsLayout L = ws_layout(*p);
   if (ws_bytes < L.total) return SPARGE_EWORKSPACE;
-  if ((st = select_device(q)) != SPARGE_OK) return st;
+  DeviceScope dev;
+  if ((st = dev.enter(q)) != SPARGE_OK) return st;
   AttnPtrs x{};
   x.q = p->qk_int8 ? static_cast<const void*>(ws_ptr<int8_t>(ws, L.q_codes)) : q;
   x.k = p->qk_int8 ? static_cast<const void*>(ws_ptr<int8_t>(ws, L.k_codes)) : k;
@@ -256,7 +252,8 @@ sparge_status_t sparge_attn_fwd(const sparge_params_t* p, const void* q, const v
 
 sparge_status_t sparge_device_status(void* ws, cudaStream_t stream) {
   if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & 255u)) return SPARGE_EINVAL;
-  sparge_status_t st = select_device(ws);
+  DeviceScope dev;
+  sparge_status_t st = dev.enter(ws);
   if (st != SPARGE_OK) return st;
   if (cudaStreamSynchronize(stream) != cudaSuccess) return SPARGE_ECUDA;
   int32_t h = 0;

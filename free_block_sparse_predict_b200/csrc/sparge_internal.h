@@ -28,7 +28,8 @@ struct WsLayout {
   size_t dq;        // [B, Hq, Tm] f32
   size_t dk;        // [B, Hkv, Tn] f32
   size_t kbar;      // [B, Hkv, d] f32
-  size_t kbar_part; // [B, Hkv, kKbarSlices, d] f32 partial sums of kbar
+  size_t kbar_part; // [B, Hkv, kKbarSlices, d] f64 partial sums of kbar
+  size_t k_sum64;   // [B, Hkv, Tn, d] f64 column sums of every K block
   size_t total;
   static constexpr size_t npos = ~size_t(0);
 };
@@ -54,9 +55,10 @@ inline WsLayout ws_layout(const sparge_params_t& p) {
     w.dq = take(size_t(p.B) * p.Hq * Tm * 4);
     w.dk = take(size_t(p.B) * p.Hkv * Tn * 4);
     w.kbar = take(size_t(p.B) * p.Hkv * p.d * 4);
-    w.kbar_part = take(size_t(p.B) * p.Hkv * kKbarSlices * p.d * 4);
+    w.kbar_part = take(size_t(p.B) * p.Hkv * kKbarSlices * p.d * 8);
+    w.k_sum64 = take(size_t(p.B) * p.Hkv * Tn * p.d * 8);
   } else {
-    w.q_codes = w.k_codes = w.dq = w.dk = w.kbar = w.kbar_part = WsLayout::npos;
+    w.q_codes = w.k_codes = w.dq = w.dk = w.kbar = w.kbar_part = w.k_sum64 = WsLayout::npos;
   }
   w.total = off;
   return w;
@@ -66,6 +68,44 @@ template <typename T>
 inline T* ws_ptr(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
 }
+
+// Host validation of a parameter set shared by every entry point that takes
+// one: SPARGE_OK, SPARGE_EINVAL or SPARGE_EUNSUPPORTED (sparge_api.cu).
+sparge_status_t check_params(const sparge_params_t* p);
+
+// Makes the device that owns a pointer current for one entry point and puts
+// the caller's current device back when it leaves scope.
+class DeviceScope {
+ public:
+  DeviceScope() = default;
+  DeviceScope(const DeviceScope&) = delete;
+  DeviceScope& operator=(const DeviceScope&) = delete;
+  ~DeviceScope() {
+    if (prev_ >= 0) cudaSetDevice(prev_);
+  }
+  // SPARGE_EINVAL when ptr is not device (or managed) memory.
+  sparge_status_t enter(const void* ptr) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
+      cudaGetLastError();
+      return SPARGE_EINVAL;
+    }
+    if (a.type != cudaMemoryTypeDevice && a.type != cudaMemoryTypeManaged) return SPARGE_EINVAL;
+    int cur = -1;
+    if (cudaGetDevice(&cur) != cudaSuccess) return SPARGE_ECUDA;
+    if (cur != a.device) {
+      if (cudaSetDevice(a.device) != cudaSuccess) return SPARGE_ECUDA;
+      prev_ = cur;
+    }
+    device_ = a.device;
+    return SPARGE_OK;
+  }
+  int device() const { return device_; }
+
+ private:
+  int prev_ = -1;
+  int device_ = -1;
+};
 
 // ------------------------------------------------------------- predict.cu
 struct PredictPtrs {
@@ -80,7 +120,8 @@ struct PredictPtrs {
   float* dq;
   float* dk;
   float* kbar;
-  float* kbar_part;
+  double* kbar_part;
+  double* ksum64;
   uint8_t* mask;
   int32_t* kv_idx;
   int32_t* kv_cnt;

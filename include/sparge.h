@@ -20,6 +20,8 @@
  *              workspaces.
  *   Streams    Every call is asynchronous on the given stream; no call
  *              synchronises except sparge_device_status.
+ *   Devices    A call runs on the device that owns its (first) device
+ *              pointer and leaves the caller's current device as it was.
  *   Errors     Arguments are validated on the host before any launch:
  *              SPARGE_EINVAL (bad pointer, size or hyper-parameter),
  *              SPARGE_EUNSUPPORTED (valid but not implemented, e.g. d = 96,
@@ -113,7 +115,9 @@ sparge_status_t sparge_hilbert_permute(const void* x, void* y, int32_t B, int32_
                                        cudaStream_t stream);
 
 /* The inverse: x[b, h, perm[p], :] = y[b, h, p, :], under the same rules (a
- * row whose entry lies outside [0, N) is not written). */
+ * row whose entry lies outside [0, N) is not written).  perm should be a
+ * permutation: if two in-range entries are equal, both source rows are
+ * written to the same destination row and which one remains is unspecified. */
 sparge_status_t sparge_inverse_permute(const void* y, void* x, int32_t B, int32_t H, int32_t N,
                                        int32_t d, sparge_dtype_t dtype, const int32_t* perm,
                                        cudaStream_t stream);
@@ -161,21 +165,27 @@ sparge_status_t sparge_predict_select(const sparge_params_t* p, uint8_t* mask, i
  * + align256(B*Hq*T_m*4) + align256(B*Hkv*T_n*4) <= 32 MiB, else the call
  * returns SPARGE_EWORKSPACE (align256 rounds up to a multiple of 256).
  * qk_int8 = 1 returns SPARGE_EUNSUPPORTED (the INT8 codes must outlive the
- * call); parameter sets that sparge_workspace_bytes rejects return
- * SPARGE_EINVAL.  The first call on each device looks up the array's device
- * address there (cudaGetSymbolAddress), so make that first call before any
- * stream capture.  The call allocates nothing.  All calls share the array and
- * it keeps the last call's contents; each call rewrites every region it reads,
- * so nothing has to be cleared, but calls whose kernels overlap on the GPU
- * (unordered streams) race on it. */
+ * call); otherwise a parameter set gets the same status as from
+ * sparge_predict_mask (SPARGE_EINVAL or SPARGE_EUNSUPPORTED).  The first call
+ * on each device looks up the array's device address there
+ * (cudaGetSymbolAddress), so make that first call before any stream capture.
+ * The call allocates nothing.  All calls share the array and it keeps the
+ * last call's contents; each call rewrites every region it reads, so nothing
+ * has to be cleared, but calls whose kernels overlap on the GPU (unordered
+ * streams) race on it.  The predictor has no device-side waits, so these
+ * calls leave no device status to read (there is no workspace to hold one). */
 sparge_status_t sparge_predict_mask_noalloc(const sparge_params_t* p, const void* q,
                                             const void* k, uint8_t* mask, int32_t* kv_idx,
                                             int32_t* kv_cnt, float* s_q, float* s_k,
                                             cudaStream_t stream);
 
 /* Compacts a caller-built mask [B, Hq, T_m, T_n] (uint8, nonzero = keep) into
- * the kv_idx / kv_cnt skip list sparge_attn_fwd consumes.  Causal-future
- * blocks are kept if the mask keeps them (the attention masks them anyway). */
+ * the kv_idx / kv_cnt skip list sparge_attn_fwd consumes: Algorithm 1 step 9
+ * visits, for query block i, the key blocks j with M_g[i, j] = 1 in ascending
+ * order, and Eq. 2 skips the others; this is that visiting order.  Causal-
+ * future blocks are kept if the mask keeps them (the attention masks them
+ * anyway).  Outputs as for sparge_predict_mask; errors as for every entry
+ * point (SPARGE_EINVAL for null or misaligned pointers). */
 sparge_status_t sparge_mask_compact(const sparge_params_t* p, const uint8_t* mask,
                                     int32_t* kv_idx, int32_t* kv_cnt, cudaStream_t stream);
 

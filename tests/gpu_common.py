@@ -124,7 +124,8 @@ def ws_regions(p):
         for name, nbytes in (("q_codes", p.B * p.Hq * p.N * p.d),
                              ("k_codes", p.B * p.Hkv * p.N * p.d), ("dq", p.B * p.Hq * Tm * 4),
                              ("dk", p.B * p.Hkv * Tn * 4), ("kbar", p.B * p.Hkv * p.d * 4),
-                             ("kbar_part", p.B * p.Hkv * 32 * p.d * 4)):
+                             ("kbar_part", p.B * p.Hkv * 32 * p.d * 8),
+                             ("k_sum64", p.B * p.Hkv * Tn * p.d * 8)):
             out[name] = off
             off += al(nbytes)
     return out
@@ -153,3 +154,45 @@ def tile_rows(w, tiles):
     for (b, h, i) in tiles:
         sel[b, h, i * w.bq:min(w.N, (i + 1) * w.bq)] = True
     return sel
+
+
+# Bounds on the mask comparison.  The ambiguity bands (1e-4 of cumulative
+# mass around tau, 1e-4 around theta) flag about 2e-4 of the visible blocks
+# on the sparse settings; a band too wide to be honest would flag far more.
+AMB_CUT_MAX_FRAC = 1e-3       # entries flagged near the TopCdf cut
+DIFF_MAX_FRAC = 1e-4          # entries where the GPU and the oracle differ
+
+
+def check_mask(M, pr, label):
+    """GPU mask M [B,Hq,Tm,Tn] bool against the oracle's prediction: equal
+    outside the ambiguous entries, with the counts printed and bounded."""
+    B, Hq = M.shape[:2]
+    vis = int(pr["visible"].sum()) * B * Hq
+    diff = M != pr["M"]
+    bad = diff & ~pr["amb"]
+    n_cut, n_th = int(pr["amb_cut"].sum()), int(pr["amb_theta"].sum())
+    d_cut, d_th = int((diff & pr["amb_cut"]).sum()), int((diff & pr["amb_theta"]).sum())
+    print(f"[mask {label}] visible {vis}, kept {int(M.sum())}: ambiguous near the cut "
+          f"{n_cut}, in rows/columns near theta {n_th}; differing {int(diff.sum())} "
+          f"(near the cut {d_cut}, near theta {d_th})")
+    assert not bad.any(), f"{int(bad.sum())} mismatches outside the ambiguous entries, " \
+                          f"first {np.argwhere(bad)[:3]}"
+    assert n_cut <= AMB_CUT_MAX_FRAC * vis, (n_cut, vis)
+    assert d_cut <= DIFF_MAX_FRAC * vis, (d_cut, vis)
+    return {"visible": vis, "amb_cut": n_cut, "amb_theta": n_th, "diff": int(diff.sum())}
+
+
+def report_lambda(ost, label, rows=None):
+    """Prints the lambda decisions within 1e-3 of the threshold and the rows
+    they exclude from the comparison.  Bounded to 1e-3 of all (slice, block)
+    decisions the oracle took, and to half of the compared rows (a long tile
+    takes tens of thousands of decisions, each of which excludes 32 rows)."""
+    near = ost["near_rows"] if rows is None else ost["near_rows"] & rows
+    n_rows = int(near.sum())
+    total = int(near.size if rows is None else rows.sum())
+    decisions = 4 * int(ost["qk_blocks"])
+    print(f"[lambda {label}] near-threshold decisions {ost['near_lambda']} of {decisions}, "
+          f"rows excluded {n_rows} of {total}")
+    assert ost["near_lambda"] <= 1e-3 * max(decisions, 1), (ost["near_lambda"], decisions)
+    assert n_rows <= 0.5 * max(total, 1), (n_rows, total)
+    return n_rows

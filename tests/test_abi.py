@@ -59,7 +59,8 @@ def test_workspace_bytes_covers_every_region(native):
     Tm, Tn = N // 128, N // 64
     floor = (B * Hq * Tm * d * 4 + B * Hkv * Tn * d * 4      # pooled means
              + B * Hkv * N * d * 2                           # fp16 V
-             + B * (Hq + Hkv) * N * d)                       # INT8 codes
+             + B * (Hq + Hkv) * N * d                        # INT8 codes
+             + B * Hkv * Tn * d * 8)                         # float64 K block sums (kbar)
     assert floor <= n <= floor + 16 * 1024 * 1024
     assert L.sparge_workspace_bytes(ctypes.byref(_params(native, qk_int8=0, io_dtype=0,
                                                           o_dtype=0))) < n

@@ -21,16 +21,27 @@ from synth import get_workload  # noqa: E402
 
 
 def test_pool_bytes_hand_count_128k_int8():
+    # the survey's algorithmic bytes of the pooling stage: one read of Q and K,
+    # the block means and self-similarities, and with INT8 the codes and scales
     w = get_workload("llm_128k")
     q = 32 * 131072 * 128 * 2            # read Q (bf16)
     k = 8 * 131072 * 128 * 2             # read K
     means = (32 * 1024 + 8 * 2048) * (128 + 1) * 4   # block means and self-similarities
     q_codes = 32 * 131072 * 128 + 32 * 1024 * 4      # Q codes and their scales
-    kbar = 8 * 2048 * 128 * 4            # k-bar from the K block means
-    k_again = 8 * 131072 * 128 * 2       # second read of K
     k_codes = 8 * 131072 * 128 + 8 * 2048 * 4        # K codes and their scales
-    assert bench.pool_bytes(w) == q + k + means + q_codes + kbar + k_again + k_codes
-    assert bench.pool_bytes(w) == 2_315_649_024
+    assert bench.pool_bytes(w) == q + k + means + q_codes + k_codes
+    assert bench.pool_bytes(w) == 2_038_824_960
+    # not counted: the second read of K and the float64 block sums of kbar
+    assert bench.pool_extra_bytes(w) == 8 * 131072 * 128 * 2 + 2 * 8 * 2048 * 128 * 8
+
+
+def test_attention_peak_weights_each_dtype():
+    peaks = {"bf16_tflops_sustained": 1000.0, "bf16_tflops": 1200.0}
+    w8 = get_workload("llm_128k")
+    # equal flops in INT8 (2000) and fp16 (1000): 2 / (1/2000 + 1/1000)
+    assert bench.attn_peak_tflops(w8, peaks, 10, 10) == pytest.approx(4000.0 / 3.0)
+    assert bench.attn_peak_tflops(w8, peaks, 10, 10, key="bf16_tflops") == pytest.approx(1600.0)
+    assert bench.attn_peak_tflops(get_workload("llm_32k"), peaks, 10, 10) == 1000.0
 
 
 def test_pool_bytes_without_int8_is_one_read_plus_means():
@@ -67,6 +78,11 @@ def test_reference_arm_prints_one_json_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["value"] == d["value"]
     assert d["higher_is_better"] is True and d["n_gpus"] == 1
+    # the same config object as the native arm, and a time it actually measured
+    w = get_workload("tiny")
+    from synth import make_qkv
+    assert d["config"] == bench.workload_config(w, 1, bench._bytes(make_qkv(w)))
+    assert d["ms_per_step"] * d["steps"] < 600e3
 
 
 def test_profiled_traffic_only_for_the_profiled_workload(tmp_path):

@@ -54,6 +54,32 @@ def test_noalloc_predictor_matches_workspace_predictor_twice():
         _same(ref, got, p)
 
 
+def test_noalloc_second_call_same_shape_new_inputs():
+    """Two calls with the same parameters and different inputs: a scratch
+    region the second call failed to rewrite would still hold the first
+    call's values, which would be right for the first inputs only."""
+    w, _ = workload("llm_32k", N=8192, Hq=8, Hkv=2)
+    p = params_for(w)
+    from synth import make_qkv
+    for seed in (1, 2):
+        t = make_qkv(w, seed=seed)
+        q, k = to_dev(t["q"], w.dtype), to_dev(t["k"], w.dtype)
+        got = _without_workspace(p, q, k)
+        ref = _with_workspace(p, q, k)
+        torch.cuda.synchronize()
+        _same(ref, got, p)
+
+
+def test_noalloc_leaves_the_current_device_alone():
+    w, t = workload("tiny")
+    p = params_for(w)
+    q, k = to_dev(t["q"], w.dtype), to_dev(t["k"], w.dtype)
+    before = torch.cuda.current_device()
+    _without_workspace(p, q, k)
+    torch.cuda.synchronize()
+    assert torch.cuda.current_device() == before
+
+
 def test_noalloc_rejects_what_it_cannot_hold():
     w, t = workload("llm_32k", N=4096, Hq=2, Hkv=1)
     q, k = to_dev(t["q"], w.dtype), to_dev(t["k"], w.dtype)
@@ -71,3 +97,10 @@ def test_noalloc_rejects_what_it_cannot_hold():
     with pytest.raises(fb.SpargeError) as e:
         fb.sparge_predict_mask_noalloc(params_for(w, qk_int8=True), q, k, *outs)
     assert e.value.code == 2
+    # a parameter set the workspace predictor calls unsupported (d = 96) gets
+    # the same status here
+    odd = params_for(w)
+    odd.d = 96
+    code = fb._native.lib().sparge_predict_mask_noalloc(ctypes.byref(odd), P(q), P(k),
+                                                        *[P(x) for x in outs], None)
+    assert code == 2
