@@ -261,7 +261,9 @@ def predict_mask(Q: np.ndarray, K: np.ndarray, bq: int, bk: int, tau: float, the
 
     Returns a dict with M [B,Hq,Tm,Tn] bool, q, k, s_q, s_k, S_hat and the
     ambiguity map amb [B,Hq,Tm,Tn] bool (entries whose decision lies within the
-    stated margins of a cut and may legitimately differ in float32).
+    stated margins of a cut and may legitimately differ in float32), split into
+    amb_theta (rows and columns whose self-similarity is within amb_sim of
+    theta) and amb_cut (entries near the TopCdf cut).
     """
     B, Hq, N, d = Q.shape
     Hkv = K.shape[1]
@@ -281,6 +283,7 @@ def predict_mask(Q: np.ndarray, K: np.ndarray, bq: int, bk: int, tau: float, the
             s_k[b, h] = block_cossim(K[b, h], bk)
     M = np.zeros((B, Hq, Tm, Tn), dtype=bool)
     amb = np.zeros((B, Hq, Tm, Tn), dtype=bool)
+    amb_theta = np.zeros((B, Hq, Tm, Tn), dtype=bool)
     S_hat = np.zeros((B, Hq, Tm, Tn))
     for b in range(B):
         for h in range(Hq):
@@ -308,12 +311,13 @@ def predict_mask(Q: np.ndarray, K: np.ndarray, bq: int, bk: int, tau: float, the
                     a[np.flatnonzero(fin)[near_cut | near_tie]] = True
             # an entry whose column is near theta can flip in or out of TopCdf
             # and of the fix rule
-            amb[b, h][:, np.abs(s_k[b, hk] - theta) <= amb_sim] = True
-            amb[b, h][np.abs(s_q[b, h] - theta) <= amb_sim, :] = True
+            amb_theta[b, h][:, np.abs(s_k[b, hk] - theta) <= amb_sim] = True
+            amb_theta[b, h][np.abs(s_q[b, h] - theta) <= amb_sim, :] = True
             M[b, h] = apply_fix_rule(Mt, s_q[b, h], s_k[b, hk], theta, vis)
+            amb_theta[b, h] &= vis
             amb[b, h] &= vis
-    return {"M": M, "amb": amb, "q": qm, "k": km, "s_q": s_q, "s_k": s_k, "S_hat": S_hat,
-            "visible": vis}
+    return {"M": M, "amb": amb | amb_theta, "amb_theta": amb_theta, "amb_cut": amb & ~amb_theta,
+            "q": qm, "k": km, "s_q": s_q, "s_k": s_k, "S_hat": S_hat, "visible": vis}
 
 
 def mask_compact(M: np.ndarray):
