@@ -765,77 +765,94 @@ def _measure(w, steps=3, warmup=2, perm=None, want_output=False, seed=0, tensors
     return out, extra
 
 
+SWEEP_LENGTHS = (8192, 16384, 32768, 65536, 131072)
+SWEEP_TAUS = (0.3, 0.5, 0.7, 0.8, 0.9, 0.95, 0.99, 1.0)
+
+
+def permutation_tables(w, rng_seed=0):
+    """Token orders of the permutation sweep on a grid workload: random,
+    row-major (the stored order), time-major, and the Hilbert curve (from the
+    library, which matches the oracle's curve bit for bit)."""
+    T, H, W = w.grid
+    P, L = w.prefix_len, T * H * W
+    rng = np.random.default_rng(rng_seed)
+    lin = np.arange(L)
+    tt, rem = np.divmod(lin, H * W)
+    yy, xx = np.divmod(rem, W)
+    return {
+        "random": np.concatenate([np.arange(P), P + rng.permutation(L)]),
+        "rowmajor": np.arange(w.N),
+        "timemajor": np.concatenate([np.arange(P), P + np.lexsort((tt, xx, yy))]),
+        "hilbert": None,
+    }
+
+
+def sweep_points(kind, base):
+    """The configurations one sweep visits, as (label, workload, permutation
+    name or None): Table 6's split (paper review, section 六) at the
+    configuration's theta and at lower ones where blocks are selective; the
+    length sweep; the tau sweep with every block selective (theta = -1), the
+    speed-against-sparsity curve; and the token orders of Table 4."""
+    pts = []
+    if kind == "table6":
+        for theta in (base.theta, 0.3, 0.0):
+            for name, over in (("only_mg", {"lam": float("-inf")}), ("only_mpv", {"theta": 2.0}),
+                               ("both", {})):
+                pts.append((f"{name} theta={theta}", base.replace(**{"theta": theta, **over}),
+                            None))
+    elif kind == "length":
+        for n in SWEEP_LENGTHS:
+            pts.append((f"N={n}", base.replace(N=n), None))
+    elif kind == "tau":
+        for tau in SWEEP_TAUS:
+            pts.append((f"tau={tau}", base.replace(tau=tau, theta=-1.0), None))
+    elif kind == "permutation":
+        for name in ("random", "rowmajor", "timemajor", "hilbert"):
+            for theta in (base.theta, 0.3):
+                pts.append((f"{name} theta={theta}", base.replace(theta=theta), name))
+    return pts
+
+
 def run_sweep(args):
     import torch
     kind = args.sweep
     base = _workload(args)
-    lines = []
-    if kind == "table6":
-        # Table 6 of the paper review: only M_g (lambda = -inf), only M_pv
-        # (theta > 1: every block computed), and both; at the configuration's
-        # theta and at lower theta values that make blocks selective
-        for theta in (base.theta, 0.3, 0.0):
-            for name, over in (("only_mg", {"lam": float("-inf")}), ("only_mpv", {"theta": 2.0}),
-                               ("both", {})):
-                w = base.replace(**{"theta": theta, **over})
-                r, _ = _measure(w)
-                r.update(sweep="table6", strategy=name, theta_setting=theta)
-                lines.append(r)
-    elif kind == "length":
-        for n in (8192, 16384, 32768, 65536, 131072):
-            w = base.replace(N=n)
-            r, _ = _measure(w)
-            r.update(sweep="length")
-            lines.append(r)
-    elif kind == "tau":
-        # speed against sparsity (Fig. 9 of the paper review) with every block
-        # selective (theta = -1) so that TopCdf alone sets the block mask
-        for tau in (0.3, 0.5, 0.7, 0.8, 0.9, 0.95, 0.99, 1.0):
-            w = base.replace(tau=tau, theta=-1.0)
-            r, _ = _measure(w)
-            r.update(sweep="tau")
-            lines.append(r)
-    elif kind == "permutation":
-        # Table 4 of the paper review on the synthetic video grid: block
-        # self-similarity, L1 error against dense attention, and sparsity
+    if kind == "permutation" and not base.grid:
+        base = get_workload("video_dit")
+    dev = torch.device("cuda", 0)
+    sampler = ClockSampler(_gpu_uuid(torch, dev))
+    t_base = make_qkv(base, seed=0)
+    perms = permutation_tables(base) if kind == "permutation" else {}
+    if kind == "permutation":
         import free_block_sparse_predict_b200 as fb
-        w = get_workload(args.workload if args.workload in ("image_dit", "video_dit")
-                         else "video_dit")
-        t = make_qkv(w, seed=0)
-        T, H, W = w.grid
-        P, L = w.prefix_len, T * H * W
-        rng = np.random.default_rng(0)
-        lin = np.arange(L)
-        tt, rem = np.divmod(lin, H * W)
-        yy, xx = np.divmod(rem, W)
-        perms = {
-            "random": np.concatenate([np.arange(P), P + rng.permutation(L)]),
-            "rowmajor": np.arange(w.N),
-            "timemajor": np.concatenate([np.arange(P), P + np.lexsort((tt, xx, yy))]),
-        }
-        dev = torch.device("cuda", 0)
-        hp = torch.empty(w.N, dtype=torch.int32, device=dev)
+        T, H, W = base.grid
+        hp = torch.empty(base.N, dtype=torch.int32, device=dev)
         hws = torch.zeros(fb.sparge_hilbert_workspace_bytes(T, H, W), dtype=torch.uint8,
                           device=dev)
-        fb.sparge_hilbert_index(w.N, P, T, H, W, hp, hws)
+        fb.sparge_hilbert_index(base.N, base.prefix_len, T, H, W, hp, hws)
         perms["hilbert"] = hp.cpu().numpy()
-        dense_w = w.replace(theta=2.0, lam=float("-inf"))
-        for name, perm in perms.items():
-            _, dense = _measure(dense_w, steps=1, warmup=1, perm=perm, want_output=True, tensors=t)
-            # the configuration's theta, and a lower one at which blocks can be selective
-            for theta in (w.theta, 0.3):
-                r, sp = _measure(w.replace(theta=theta), steps=3, warmup=1, perm=perm,
-                                 want_output=True, tensors=t)
-                O, O2 = dense["o"], sp["o"]
-                l1 = float((O - O2).abs().sum() / O.abs().sum())
-                nq = P // w.bq
-                nk = P // w.bk
-                r.update(sweep="permutation", permutation=name,
-                         sim_q=round(float(sp["s_q"][..., nq:].mean()), 4),
-                         sim_k=round(float(sp["s_k"][..., nk:].mean()), 4), l1=round(l1, 5))
-                lines.append(r)
-    for r in lines:
-        r["workload"] = base.name if kind != "permutation" else r.get("workload", "video_dit")
+    dense = {}
+    for label, w, pname in sweep_points(kind, base):
+        tensors = t_base if w.N == base.N else make_qkv(w, seed=0)
+        perm = perms.get(pname) if pname else None
+        sampler.start()
+        r, extra = _measure(w, perm=perm, want_output=kind == "permutation", tensors=tensors)
+        clocks = sampler.stop()
+        r.update(sweep=kind, point=label, clocks=clocks, workload=w.name)
+        if kind == "table6":
+            r.update(theta_setting=w.theta)
+        if kind == "permutation":
+            # Table 4's columns: block self-similarity and L1 against dense attention
+            if pname not in dense:
+                _, d_extra = _measure(w.replace(theta=2.0, lam=float("-inf")), steps=1, warmup=1,
+                                      perm=perm, want_output=True, tensors=tensors)
+                dense[pname] = d_extra["o"]
+            O, O2 = dense[pname], extra["o"]
+            nq, nk = w.prefix_len // w.bq, w.prefix_len // w.bk
+            r.update(permutation=pname,
+                     sim_q=round(float(extra["s_q"][..., nq:].mean()), 4),
+                     sim_k=round(float(extra["s_k"][..., nk:].mean()), 4),
+                     l1=round(float((O - O2).abs().sum() / O.abs().sum()), 5))
         print(json.dumps(r), flush=True)
 
 

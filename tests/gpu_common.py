@@ -159,8 +159,9 @@ def tile_rows(w, tiles):
 # Bounds on the mask comparison.  The ambiguity bands (1e-4 of cumulative
 # mass around tau, 1e-4 around theta) flag about 2e-4 of the visible blocks
 # on the sparse settings; a band too wide to be honest would flag far more.
-AMB_CUT_MAX_FRAC = 1e-3       # entries flagged near the TopCdf cut
-DIFF_MAX_FRAC = 1e-4          # entries where the GPU and the oracle differ
+# Small masks get a few entries of slack (a row of near-equal weights).
+AMB_CUT_MAX_FRAC, AMB_CUT_MIN = 1e-3, 16   # entries flagged near the TopCdf cut
+DIFF_MAX_FRAC, DIFF_MIN = 1e-4, 2          # entries where the GPU and the oracle differ
 
 
 def check_mask(M, pr, label):
@@ -177,8 +178,8 @@ def check_mask(M, pr, label):
           f"(near the cut {d_cut}, near theta {d_th})")
     assert not bad.any(), f"{int(bad.sum())} mismatches outside the ambiguous entries, " \
                           f"first {np.argwhere(bad)[:3]}"
-    assert n_cut <= AMB_CUT_MAX_FRAC * vis, (n_cut, vis)
-    assert d_cut <= DIFF_MAX_FRAC * vis, (d_cut, vis)
+    assert n_cut <= max(AMB_CUT_MAX_FRAC * vis, AMB_CUT_MIN), (n_cut, vis)
+    assert d_cut <= max(DIFF_MAX_FRAC * vis, DIFF_MIN), (d_cut, vis)
     return {"visible": vis, "amb_cut": n_cut, "amb_theta": n_th, "diff": int(diff.sum())}
 
 
