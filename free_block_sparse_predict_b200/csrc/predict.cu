@@ -67,12 +67,6 @@ __device__ __forceinline__ uint4 opaque(uint4 v) {
   return v;
 }
 
-__device__ __forceinline__ float fmax3(float a, float b, float c) {
-  float r;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
-  return r;
-}
-
 __device__ __forceinline__ void named_barrier(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
@@ -106,10 +100,9 @@ __device__ __forceinline__ float absmax2_value(uint32_t acc) {
 }
 
 // rint(x / delta) of eight values by the IEEE division itself, as the bits
-// of q + 1.5 * 2^23 (the code is their low byte).  Out of line: it runs for
-// about one call in a thousand, and inlined into every unrolled row of the
-// pooling kernel it made the kernel's code too large to stay in the
-// instruction cache.
+// of q + 1.5 * 2^23 (the code is their low byte).  Out of line: it runs only
+// for a subnormal delta, and inlined into every unrolled row of the pooling
+// kernel it would make the kernel's code too large for the instruction cache.
 __device__ __noinline__ uint2 codes8_exact(float x0, float x1, float x2, float x3, float x4,
                                            float x5, float x6, float x7, float delta) {
   constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
@@ -125,40 +118,37 @@ __device__ __noinline__ uint2 codes8_exact(float x0, float x1, float x2, float x
 }
 
 // Eight INT8 codes rint(x / delta): round half to even of the IEEE float32
-// quotient.  Fast path: t = x * inv with inv = 1/delta correctly rounded,
-// then t + 1.5 * 2^23 rounds t to the nearest integer, ties to even, exactly
-// (|t| < 2^22), and the code is the low byte of that sum's bits, two's
-// complement included.  t differs from the quotient fl(x / delta) by less than
-// 1.9e-5 (|x / delta| <= 127.00001, two roundings of 2^-24 relative each, and
-// the quotient's own half ulp of 2^-18), so rint(t) is rint(fl(x / delta))
-// unless t lies within 2^-14 of a half-integer.  Those take the slow path:
-// the IEEE division itself.  The products and sums are explicit .rn
-// instructions, so none is fused.
+// quotient.  The quotient comes from the reciprocal y = RN(1/delta) by
+// Markstein's final correction step for division with a fused multiply-add:
+// q0 = RN(x y), r = RN(x - q0 delta), q = RN(q0 + r y), which is the correctly
+// rounded x / delta (it is the last step of FMA-based IEEE division; checked
+// here against exact rational arithmetic on bf16 and float32 inputs, on
+// quotients at and next to half-integers, and by the bit-exact GPU tests).
+// Then q + 1.5 * 2^23 rounds q to the nearest integer, ties to even, exactly
+// (|q| < 2^22), and the code is the low byte of that sum's bits, two's
+// complement included.  Every step is an explicit .rn instruction on packed
+// pairs, so nothing is fused or reordered.  A subnormal delta, whose
+// reciprocal overflows, takes the IEEE division instead.
 __device__ __forceinline__ uint2 codes8(const uint64_t (&x2)[4], float inv, float delta,
                                         bool exact_only) {
   constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
-  constexpr float kNear = 0.5f - 1.0f / 16384.0f;
-  const uint64_t inv2 = pack2(inv, inv), mg2 = pack2(kMagic, kMagic);
-  uint32_t bits[8];
-  float dmax = 0.f;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint64_t t2 = mul2(x2[i], inv2);
-    const uint64_t r2 = add2(t2, mg2);
-    const uint64_t d2 = sub2(t2, sub2(r2, mg2));  // t - rint(t), exact
-    float r0, r1, d0, d1;
-    unpack2(r2, r0, r1);
-    unpack2(d2, d0, d1);
-    bits[2 * i] = __float_as_uint(r0);
-    bits[2 * i + 1] = __float_as_uint(r1);
-    dmax = fmax3(dmax, fabsf(d0), fabsf(d1));
-  }
-  // (a NaN distance fails the test and also takes the exact path)
-  if (exact_only || !(dmax <= kNear)) {
+  if (exact_only) {
     float v[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) unpack2(x2[i], v[2 * i], v[2 * i + 1]);
     return codes8_exact(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7], delta);
+  }
+  const uint64_t inv2 = pack2(inv, inv), nd2 = pack2(-delta, -delta), mg2 = pack2(kMagic, kMagic);
+  uint32_t bits[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint64_t q0 = mul2(x2[i], inv2);
+    const uint64_t r = fma2(q0, nd2, x2[i]);    // x - q0 delta
+    const uint64_t q = fma2(r, inv2, q0);       // q0 + r y
+    float r0, r1;
+    unpack2(add2(q, mg2), r0, r1);
+    bits[2 * i] = __float_as_uint(r0);
+    bits[2 * i + 1] = __float_as_uint(r1);
   }
   const uint32_t lo = __byte_perm(__byte_perm(bits[0], bits[1], 0x0040),
                                   __byte_perm(bits[2], bits[3], 0x0040), 0x5410);
