@@ -19,6 +19,7 @@
 
 #include <algorithm>
 #include <cfloat>
+#include <climits>
 #include <cstdint>
 
 #include "sm100_ptx.cuh"
@@ -57,6 +58,18 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
                : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
                : "l"(p));
   return r;
+}
+
+// 16 bytes global -> shared, cached in L2 only; completed by cp_async_wait.
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
 }
 
 // Same bits, but opaque to the compiler: keeps it from holding every row's
@@ -169,8 +182,12 @@ __device__ __forceinline__ double f32_to_f64_bits(float x) {
   return __hiloint2double(int(hi), 0);
 }
 
-// One warp per SLAB-row slab of a block, held in registers for the whole
-// pass, so every byte of Q and K is read from HBM exactly once per pass.
+// One warp per SLAB-row slab of a block, held in registers while the block
+// is processed, so every byte of Q and K is read from HBM exactly once per
+// pass.  The kernel is persistent: a CTA of four warps takes units of four
+// slabs (one Q block or two K blocks) in a grid-stride loop, and each warp
+// copies its slab of the next unit into its shared-memory buffer (cp.async)
+// while it works on the current one, so loads stay in flight all the time.
 // Lane (ro, c) owns the 16-byte chunk c of rows ro, ro + RPW, ...  Arithmetic
 // runs on packed fp32 pairs in two sweeps over the registers: the first takes
 // the squared row norms, the column sums of x and the exact |x| max; the
@@ -192,6 +209,11 @@ template <int D, bool BF16, int KIND, int SLAB>
 __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(PoolArgs a) {
   constexpr bool POOL = KIND != 1;
   constexpr bool SUM64 = KIND == 2;
+  // The Q pass is persistent and stages the next unit in shared memory; the
+  // two small K passes take one unit per CTA and load straight into
+  // registers (staging gains them nothing, and KIND 2's float64 sums leave no
+  // registers for the loop's state).
+  constexpr bool PERSIST = KIND == 0;
   constexpr int CH = D * 2 / 16;  // lanes per row
   constexpr int RPW = 32 / CH;    // rows per warp-wide load
   constexpr int NR = SLAB / RPW;  // rows per lane
@@ -203,33 +225,90 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
   __shared__ float part[WARPS][2 * D];
   __shared__ float pmax[WARPS];
   __shared__ double part64[SUM64 ? WARPS : 1][SUM64 ? D : 1];
+  __shared__ __align__(16) uint4 stage[PERSIST ? WARPS : 1][PERSIST ? NR : 1][32];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t gw = int64_t(blockIdx.x) * WARPS + warp;
-  const int64_t nQw = a.nQblocks * GQ;
-  const bool isQ = KIND == 0 && gw < nQw;
-  const int G = isQ ? GQ : GK;
-  const int64_t rel = isQ ? gw : gw - nQw;
-  const int64_t nb = isQ ? a.nQblocks : a.nblocks - a.nQblocks;
-  int64_t blkid = rel / G;
-  const int sub = int(rel % G);  // slab index inside the block
-  if (blkid >= nb) return;  // whole groups leave
-  if (KIND == 1) blkid = nb - 1 - blkid;
-  const int T = isQ ? a.Tm : a.Tn;
-  const int BLK = isQ ? kPoolBQ : kPoolBK;
-  const int64_t bh = blkid / T;
-  const int blk = int(blkid % T);
-  const int rows = min(BLK, a.N - blk * BLK);
-  const int srows = max(0, min(SLAB, rows - sub * SLAB));
   const int c = lane % CH, ro = lane / CH;
-  const int64_t row0 = bh * a.N + int64_t(blk) * BLK + sub * SLAB;
-  const uint16_t* src = static_cast<const uint16_t*>(isQ ? a.q : a.k) + row0 * D + c * 8;
+  const int64_t nQw = a.nQblocks * GQ;
+  const int64_t n_units = (nQw + (a.nblocks - a.nQblocks) * GK + WARPS - 1) / WARPS;
+  // the slab that this warp takes in unit u: Q blocks first, then K blocks
+  // (KIND 1 walks its K blocks last first); whole groups of G warps are
+  // either inside or past the end
+  struct Slab {
+    bool valid, isQ;
+    int64_t bh, row0;
+    int blk, sub, rows, srows;
+  };
+  // (32-bit indices: the library refuses parameter sets with 2^31 tiles or
+  // more, and the group sizes G are powers of two)
+  auto slab_of = [&](int64_t u) {
+    Slab sl;
+    const int64_t gw64 = u * WARPS + warp;
+    const int gw = gw64 < INT32_MAX ? int(gw64) : INT32_MAX;
+    const int nqw = int(nQw);
+    sl.isQ = KIND == 0 && gw < nqw;
+    const int lg = sl.isQ ? (GQ == 4 ? 2 : GQ == 2 ? 1 : 0) : (GK == 2 ? 1 : 0);
+    const int rel = sl.isQ ? gw : gw - nqw;
+    const int nb = int(sl.isQ ? a.nQblocks : a.nblocks - a.nQblocks);
+    int bid = rel >> lg;
+    sl.sub = rel & ((1 << lg) - 1);
+    sl.valid = u < n_units && bid < nb;
+    if (KIND == 1) bid = nb - 1 - bid;
+    const int T_ = sl.isQ ? a.Tm : a.Tn;
+    const int BLK_ = sl.isQ ? kPoolBQ : kPoolBK;
+    const int bhi = bid / T_;
+    sl.bh = bhi;
+    sl.blk = bid - bhi * T_;
+    sl.rows = min(BLK_, a.N - sl.blk * BLK_);
+    sl.srows = sl.valid ? max(0, min(SLAB, sl.rows - sl.sub * SLAB)) : 0;
+    sl.row0 = sl.bh * a.N + int64_t(sl.blk) * BLK_ + sl.sub * SLAB;
+    return sl;
+  };
+  auto prefetch = [&](const Slab& sl) {
+    if (!PERSIST) return;
+    const uint16_t* src = static_cast<const uint16_t*>(sl.isQ ? a.q : a.k) + sl.row0 * D + c * 8;
+#pragma unroll
+    for (int u = 0; u < NR; ++u) {
+      const int r = ro + u * RPW;
+      if (r < sl.srows) cp_async16(&stage[warp][u][lane], src + int64_t(r) * D);
+    }
+    cp_async_commit();
+  };
+  int64_t unit = blockIdx.x;
+  Slab cur = slab_of(unit);
+  prefetch(cur);
+  for (; unit < n_units; unit += gridDim.x) {
+  cp_async_wait_all();
+  if (!cur.valid) {  // past the end: only the next unit's copies
+    if (!PERSIST) break;
+    cur = slab_of(unit + gridDim.x);
+    prefetch(cur);
+    continue;
+  }
+  const bool isQ = cur.isQ;
+  const int G = isQ ? GQ : GK;
+  const int sub = cur.sub;
+  const int T = isQ ? a.Tm : a.Tn;
+  const int64_t bh = cur.bh;
+  const int blk = cur.blk;
+  const int rows = cur.rows;
+  const int srows = cur.srows;
+  const int64_t row0 = cur.row0;
 
   uint4 raw[NR];
+  if constexpr (PERSIST) {
 #pragma unroll
-  for (int u = 0; u < NR; ++u) {
-    const int r = ro + u * RPW;
-    raw[u] = r < srows ? ld_stream(src + int64_t(r) * D) : make_uint4(0, 0, 0, 0);
+    for (int u = 0; u < NR; ++u) {
+      const int r = ro + u * RPW;
+      raw[u] = r < srows ? stage[warp][u][lane] : make_uint4(0, 0, 0, 0);
+    }
+  } else {
+    const uint16_t* src = static_cast<const uint16_t*>(isQ ? a.q : a.k) + row0 * D + c * 8;
+#pragma unroll
+    for (int u = 0; u < NR; ++u) {
+      const int r = ro + u * RPW;
+      raw[u] = r < srows ? ld_stream(src + int64_t(r) * D) : make_uint4(0, 0, 0, 0);
+    }
   }
   uint64_t nkb2[4];  // -kbar of this lane's 8 columns, as pairs
   if (KIND == 1) {
@@ -241,13 +320,13 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
   float sx[8], su[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) sx[e] = su[e] = 0.f;
+  double s64[SUM64 ? 8 : 1];  // float64 column sums (KIND 2)
+#pragma unroll
+  for (int e = 0; e < (SUM64 ? 8 : 1); ++e) s64[e] = 0.0;
   float amax = 0.f;
   float inv_own[R];
   const int group_base = lane & ~(CH - 1);
   const int w0 = warp - sub;
-  double s64[SUM64 ? 8 : 1];  // float64 column sums (KIND 2)
-#pragma unroll
-  for (int e = 0; e < (SUM64 ? 8 : 1); ++e) s64[e] = 0.0;
   if (POOL) {
     // ---- pass 1: squared row norms (one value per row), column sums of x,
     // and the exact |x| max on the raw 16-bit halves
@@ -291,8 +370,8 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
 #pragma unroll
     for (int t = 0; t < R; ++t) inv_own[t] = v[t] > 0.f ? rsqrtf(v[t]) : 0.f;
     if (SUM64) {
-      // a sweep of its own, once the row norms no longer hold registers;
-      // rows past the block are zero and add nothing
+      // float64 column sums in a sweep of their own, once the row norms no
+      // longer hold registers; rows past the block are zero and add nothing
 #pragma unroll
       for (int u = 0; u < NR; ++u) {
         const uint4 rw = opaque(raw[u]);
@@ -320,6 +399,8 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
       }
     }
   }
+  // every loaded register has been read: the buffer takes the next unit
+  if (PERSIST) prefetch(slab_of(unit + gridDim.x));
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   if (POOL) {
@@ -435,6 +516,9 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
       }
       if (lane == 0) (isQ ? a.s_q : a.s_k)[bh * T + blk] = uu / (float(rows) * float(rows));
     }
+  }
+  if (!PERSIST) break;
+  cur = slab_of(unit + gridDim.x);
   }
 }
 
@@ -723,6 +807,26 @@ __global__ void compact_kernel(const uint8_t* mask, int32_t* kv_idx, int32_t* kv
   if (lane == 0) kv_cnt[r] = cnt;
 }
 
+// Persistent pooling grid: four CTAs per SM (the kernel's occupancy), no more
+// than there are units of work (one CTA per unit for the K passes).  The shared-memory carveout is set to its
+// maximum so that four CTAs' slab buffers fit.
+template <int D, bool BF16, int KIND, int SLAB>
+cudaError_t launch_pool(const PoolArgs& pa, int64_t warps, cudaStream_t s) {
+  int dev = 0, sms = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(pool_kernel<D, BF16, KIND, SLAB>,
+                           cudaFuncAttributePreferredSharedMemoryCarveout,
+                           int(cudaSharedmemCarveoutMaxShared));
+  if (e != cudaSuccess) return e;
+  const int64_t units = cdiv(warps, kPoolThreads / 32);
+  const int64_t ctas =
+      KIND != 0 ? units : std::max<int64_t>(1, std::min<int64_t>(units, int64_t(sms) * kPoolMinBlocks));
+  pool_kernel<D, BF16, KIND, SLAB><<<unsigned(ctas), kPoolThreads, 0, s>>>(pa);
+  return cudaGetLastError();
+}
+
 template <int D, bool BF16>
 cudaError_t pool_impl(const sparge_params_t& p, const PredictPtrs& x, cudaStream_t s) {
   if (p.bq != kPoolBQ || p.bk != kPoolBK) return cudaErrorInvalidValue;
@@ -747,13 +851,10 @@ cudaError_t pool_impl(const sparge_params_t& p, const PredictPtrs& x, cudaStream
   pa.status = x.status;
   cudaError_t e;
   constexpr int SLAB = D == 128 ? 32 : 64;  // 8 KB of bf16/f16 per warp
-  constexpr int64_t warps_per_cta = kPoolThreads / 32;
   constexpr int64_t GQ = kPoolBQ / SLAB, GK = kPoolBK / SLAB;
   if (x.k_codes == nullptr) {
     // one pass over Q then K blocks
-    const int64_t w0 = pa.nQblocks * GQ + nK * GK;
-    pool_kernel<D, BF16, 0, SLAB><<<unsigned(cdiv(w0, warps_per_cta)), kPoolThreads, 0, s>>>(pa);
-    return cudaGetLastError();
+    return launch_pool<D, BF16, 0, SLAB>(pa, pa.nQblocks * GQ + nK * GK, s);
   }
   if constexpr (D != 128) {
     return cudaErrorInvalidValue;  // the INT8 path exists for d = 128 only
@@ -765,8 +866,7 @@ cudaError_t pool_impl(const sparge_params_t& p, const PredictPtrs& x, cudaStream
   ka.nQblocks = 0;
   ka.nblocks = nK;
   ka.ksum64 = x.ksum64;
-  pool_kernel<D, BF16, 2, SLAB><<<unsigned(cdiv(nK * GK, warps_per_cta)), kPoolThreads, 0, s>>>(ka);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = launch_pool<D, BF16, 2, SLAB>(ka, nK * GK, s)) != cudaSuccess) return e;
   const unsigned BHk = unsigned(int64_t(p.B) * p.Hkv);
   kbar_partial_kernel<D><<<BHk * kKbarSlices, D, 0, s>>>(x.ksum64, x.kbar_part, int32_t(Tn));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -776,13 +876,10 @@ cudaError_t pool_impl(const sparge_params_t& p, const PredictPtrs& x, cudaStream
   ca.kbar = x.kbar;
   ca.k_codes = x.k_codes;
   ca.dk = x.dk;
-  pool_kernel<D, BF16, 1, SLAB><<<unsigned(cdiv(nK * GK, warps_per_cta)), kPoolThreads, 0, s>>>(ca);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = launch_pool<D, BF16, 1, SLAB>(ca, nK * GK, s)) != cudaSuccess) return e;
   PoolArgs qa = pa;
   qa.nblocks = qa.nQblocks;
-  pool_kernel<D, BF16, 0, SLAB>
-      <<<unsigned(cdiv(qa.nQblocks * GQ, warps_per_cta)), kPoolThreads, 0, s>>>(qa);
-  return cudaGetLastError();
+  return launch_pool<D, BF16, 0, SLAB>(qa, qa.nQblocks * GQ, s);
   }
 }
 
