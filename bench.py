@@ -262,7 +262,7 @@ def run_native(args, rank, world, local_rank):
         if timing:
             timing[0].record(stream)
         fb.sparge_predict_pool(prm, qs, ks, ws, stream)
-        n += 5 if w.qk_int8 else 1
+        n += 4 if w.qk_int8 else 1
         if timing:
             timing[1].record(stream)
         fb.sparge_predict_select(prm, mask, idx, cnt, None, None, ws, stream)

@@ -8,7 +8,7 @@
 //                   With INT8 it also quantises Q per block (Algorithm 1 step 2).
 //   pool_kernel<.., 2>  with INT8, the pooling pass over K alone, which also
 //                   writes each K block's float64 column sums;
-//   kbar_*_kernel   per-head mean of K from them (K smoothing);
+//   kbar_kernel     per-head mean of K from them (K smoothing);
 //   pool_kernel<.., 1>  per-block INT8 of K - kbar (second pass over K).
 //   select_kernel   per query block: S_hat = scale q_i k^T with -inf columns
 //                   (Eq. 7), row softmax, TopCdf(tau) (Eq. 8) by an exact
@@ -170,22 +170,28 @@ __device__ __forceinline__ uint2 codes8(const uint64_t (&x2)[4], float inv, floa
   return make_uint2(lo, hi);
 }
 
-// A float32 value as float64, built from its bits (the fp64 conversion unit
-// runs at a quarter of the integer rate): exponent rebiased by 1023 - 127,
-// significand moved down three places into the high word.  Exact for every
-// float32 whose low three significand bits are zero, which holds for every
-// widened bf16 or f16 value; zeros stay zero and float32 subnormals (only a
-// bf16 below 2^-126 widens to one) are flushed to zero.
-__device__ __forceinline__ double f32_to_f64_bits(float x) {
-  const uint32_t f = __float_as_uint(x), m = f & 0x7FFFFFFFu;
-  const uint32_t hi = (f & 0x80000000u) | (m >= 0x00800000u ? (m >> 3) + 0x38000000u : 0u);
+// x * 2^-896 as a float64, built from the float32 bits of x (the fp64
+// conversion unit runs at a quarter of the integer rate): the exponent field
+// is kept as it stands, so bias 127 reads as bias 1023, and the significand
+// moves down three places into the high word.  A normal x becomes the normal
+// float64 x * 2^-896 and a float32 subnormal 0.f * 2^-126 (a bf16 below
+// 2^-126) the float64 subnormal 0.f * 2^-1022, the same scaling.  Exact for
+// every finite float32 whose low three significand bits are zero, which holds
+// for every widened bf16 or f16 value.  Sums taken in this domain round
+// exactly as the unscaled float64 sums would: every partial sum below 2^-126
+// is a multiple of 2^-133 with at most seven significant bits, exact in both.
+constexpr double kF64Unscale = 0x1p896;
+__device__ __forceinline__ double f64_scaled(float x) {
+  // arithmetic shift: the sign fills bits 31..28, the mask keeps bit 31
+  const uint32_t hi = uint32_t(int32_t(__float_as_uint(x)) >> 3) & 0x8FFFFFFFu;
   return __hiloint2double(int(hi), 0);
 }
 
 // One warp per SLAB-row slab of a block, held in registers while the block
 // is processed, so every byte of Q and K is read from HBM exactly once per
-// pass.  The kernel is persistent: a CTA of four warps takes units of four
-// slabs (one Q block or two K blocks) in a grid-stride loop, and each warp
+// pass.  A CTA of four warps takes units of four slabs (one Q block or two K
+// blocks); the Q pass and the K code pass are persistent, taking units in a
+// grid-stride loop, and each warp
 // copies its slab of the next unit into its shared-memory buffer (cp.async)
 // while it works on the current one, so loads stay in flight all the time.
 // Lane (ro, c) owns the 16-byte chunk c of rows ro, ro + RPW, ...  Arithmetic
@@ -209,11 +215,11 @@ template <int D, bool BF16, int KIND, int SLAB>
 __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(PoolArgs a) {
   constexpr bool POOL = KIND != 1;
   constexpr bool SUM64 = KIND == 2;
-  // The Q pass is persistent and stages the next unit in shared memory; the
-  // two small K passes take one unit per CTA and load straight into
-  // registers (staging gains them nothing, and KIND 2's float64 sums leave no
-  // registers for the loop's state).
-  constexpr bool PERSIST = KIND == 0;
+  // The Q pass and the K code pass are persistent and stage the next unit in
+  // shared memory; the K pooling pass takes one unit per CTA and loads
+  // straight into registers (its float64 sums leave no registers for the
+  // loop's state).
+  constexpr bool PERSIST = KIND != 2;
   constexpr int CH = D * 2 / 16;  // lanes per row
   constexpr int RPW = 32 / CH;    // rows per warp-wide load
   constexpr int NR = SLAB / RPW;  // rows per lane
@@ -380,8 +386,8 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
         for (int e = 0; e < 4; ++e) {
           float x0, x1;
           unpack2(widen2<BF16>(w[e]), x0, x1);
-          s64[2 * e] += f32_to_f64_bits(x0);
-          s64[2 * e + 1] += f32_to_f64_bits(x1);
+          s64[2 * e] += f64_scaled(x0);
+          s64[2 * e + 1] += f64_scaled(x1);
         }
       }
     }
@@ -447,7 +453,7 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
   if (SUM64 && sub == 0 && ro == 0) {
     double* dst = a.ksum64 + (bh * T + blk) * D + c * 8;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) dst[e] = s64[e];
+    for (int e = 0; e < 8; ++e) dst[e] = s64[e] * kF64Unscale;
   }
   const bool quantise = KIND == 1 || (isQ && a.q_codes != nullptr);
   // delta = absmax / 127 (IEEE divide); inv = 1 / delta correctly rounded.  A
@@ -523,32 +529,35 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
 }
 
 // kbar[bh, :] = fl32((sum over the N tokens of K[bh, :, :]) / N) with the sum
-// in float64, in a fixed order: slice s of kKbarSlices adds its key blocks'
-// float64 column sums into part[bh, s, :], then one CTA per head adds the
-// slices in index order.  For 16-bit K every partial sum is exact (the
-// exponents of realistic data span far fewer than 53 bits), so the result is
-// the float64 mean rounded once to float32, whatever the order.
-template <int D>
-__global__ void __launch_bounds__(D) kbar_partial_kernel(const double* ksum, double* part,
-                                                         int32_t Tn) {
-  const int64_t bh = blockIdx.x / kKbarSlices;
-  const int sl = int(blockIdx.x % kKbarSlices), col = threadIdx.x;
-  const int per = (Tn + kKbarSlices - 1) / kKbarSlices;
-  const int j0 = sl * per, j1 = min(Tn, j0 + per);
+// in float64, in a fixed order.  One CTA per head and four adjacent columns
+// (one 32-byte sector of a row of block sums): thread t takes column t % 4
+// and the key blocks t / 4, t / 4 + 64, ...; the 64 partial sums of a column
+// are then added by a butterfly within each warp and across the warps in
+// warp order.  For 16-bit K every partial sum is exact (the exponents of
+// realistic data span far fewer than 53 bits), so the result is the float64
+// mean rounded once to float32, whatever the order.
+constexpr int kKbarCols = 4;
+__global__ void __launch_bounds__(256) kbar_kernel(const double* ksum, float* kbar, int32_t N,
+                                                   int32_t Tn, int32_t D) {
+  __shared__ double wsum[8][kKbarCols];
+  const int groups = D / kKbarCols;
+  const int64_t bh = blockIdx.x / groups;
+  const int col = (blockIdx.x % groups) * kKbarCols + (threadIdx.x % kKbarCols);
+  const int jl = threadIdx.x / kKbarCols, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const double* src = ksum + bh * Tn * D + col;
   double acc = 0.0;
-  for (int j = j0; j < j1; ++j) acc += ksum[(bh * Tn + j) * D + col];
-  part[(bh * kKbarSlices + sl) * D + col] = acc;
-}
-
-template <int D>
-__global__ void __launch_bounds__(D) kbar_final_kernel(const double* part, float* kbar,
-                                                       int32_t N) {
-  const int64_t bh = blockIdx.x;
-  const int col = threadIdx.x;
-  double s = 0.0;
-#pragma unroll 8
-  for (int sl = 0; sl < kKbarSlices; ++sl) s += part[(bh * kKbarSlices + sl) * D + col];
-  kbar[bh * D + col] = __double2float_rn(s / double(N));
+#pragma unroll 4
+  for (int j = jl; j < Tn; j += 256 / kKbarCols) acc += src[int64_t(j) * D];
+#pragma unroll
+  for (int o = kKbarCols; o < 32; o <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+  if (lane < kKbarCols) wsum[warp][lane] = acc;
+  __syncthreads();
+  if (threadIdx.x < kKbarCols) {
+    double s = wsum[0][threadIdx.x];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) s += wsum[w][threadIdx.x];
+    kbar[bh * D + col] = __double2float_rn(s / double(N));
+  }
 }
 
 // ------------------------------------------------------------------ select
@@ -808,8 +817,9 @@ __global__ void compact_kernel(const uint8_t* mask, int32_t* kv_idx, int32_t* kv
 }
 
 // Persistent pooling grid: four CTAs per SM (the kernel's occupancy), no more
-// than there are units of work (one CTA per unit for the K passes).  The shared-memory carveout is set to its
-// maximum so that four CTAs' slab buffers fit.
+// than there are units of work (one CTA per unit for the K pooling pass).  The
+// shared-memory carveout is set to its maximum so that four CTAs' slab
+// buffers fit.
 template <int D, bool BF16, int KIND, int SLAB>
 cudaError_t launch_pool(const PoolArgs& pa, int64_t warps, cudaStream_t s) {
   int dev = 0, sms = 0;
@@ -822,7 +832,7 @@ cudaError_t launch_pool(const PoolArgs& pa, int64_t warps, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int64_t units = cdiv(warps, kPoolThreads / 32);
   const int64_t ctas =
-      KIND != 0 ? units : std::max<int64_t>(1, std::min<int64_t>(units, int64_t(sms) * kPoolMinBlocks));
+      KIND == 2 ? units : std::max<int64_t>(1, std::min<int64_t>(units, int64_t(sms) * kPoolMinBlocks));
   pool_kernel<D, BF16, KIND, SLAB><<<unsigned(ctas), kPoolThreads, 0, s>>>(pa);
   return cudaGetLastError();
 }
@@ -867,10 +877,8 @@ cudaError_t pool_impl(const sparge_params_t& p, const PredictPtrs& x, cudaStream
   ka.nblocks = nK;
   ka.ksum64 = x.ksum64;
   if ((e = launch_pool<D, BF16, 2, SLAB>(ka, nK * GK, s)) != cudaSuccess) return e;
-  const unsigned BHk = unsigned(int64_t(p.B) * p.Hkv);
-  kbar_partial_kernel<D><<<BHk * kKbarSlices, D, 0, s>>>(x.ksum64, x.kbar_part, int32_t(Tn));
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  kbar_final_kernel<D><<<BHk, D, 0, s>>>(x.kbar_part, x.kbar, p.N);
+  kbar_kernel<<<unsigned(int64_t(p.B) * p.Hkv * (D / kKbarCols)), 256, 0, s>>>(
+      x.ksum64, x.kbar, p.N, int32_t(Tn), D);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   PoolArgs ca = ka;
   ca.kbar = x.kbar;

@@ -151,7 +151,6 @@ static sparge_status_t predict_common(int stages, const sparge_params_t* p, cons
     x.dq = ws_ptr<float>(ws, L.dq);
     x.dk = ws_ptr<float>(ws, L.dk);
     x.kbar = ws_ptr<float>(ws, L.kbar);
-    x.kbar_part = ws_ptr<double>(ws, L.kbar_part);
     x.ksum64 = ws_ptr<double>(ws, L.k_sum64);
   }
   x.mask = mask;

@@ -13,8 +13,6 @@ namespace sparge {
 inline int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-constexpr int kKbarSlices = 32;  // key-block slices of the two-level kbar sum
-
 // Offsets (bytes) of every region of the caller's workspace.
 struct WsLayout {
   size_t status;    // int32 status word (kernels OR/CAS error codes in)
@@ -28,7 +26,6 @@ struct WsLayout {
   size_t dq;        // [B, Hq, Tm] f32
   size_t dk;        // [B, Hkv, Tn] f32
   size_t kbar;      // [B, Hkv, d] f32
-  size_t kbar_part; // [B, Hkv, kKbarSlices, d] f64 partial sums of kbar
   size_t k_sum64;   // [B, Hkv, Tn, d] f64 column sums of every K block
   size_t total;
   static constexpr size_t npos = ~size_t(0);
@@ -55,10 +52,9 @@ inline WsLayout ws_layout(const sparge_params_t& p) {
     w.dq = take(size_t(p.B) * p.Hq * Tm * 4);
     w.dk = take(size_t(p.B) * p.Hkv * Tn * 4);
     w.kbar = take(size_t(p.B) * p.Hkv * p.d * 4);
-    w.kbar_part = take(size_t(p.B) * p.Hkv * kKbarSlices * p.d * 8);
     w.k_sum64 = take(size_t(p.B) * p.Hkv * Tn * p.d * 8);
   } else {
-    w.q_codes = w.k_codes = w.dq = w.dk = w.kbar = w.kbar_part = w.k_sum64 = WsLayout::npos;
+    w.q_codes = w.k_codes = w.dq = w.dk = w.kbar = w.k_sum64 = WsLayout::npos;
   }
   w.total = off;
   return w;
@@ -120,7 +116,6 @@ struct PredictPtrs {
   float* dq;
   float* dk;
   float* kbar;
-  double* kbar_part;
   double* ksum64;
   uint8_t* mask;
   int32_t* kv_idx;

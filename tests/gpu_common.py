@@ -124,7 +124,6 @@ def ws_regions(p):
         for name, nbytes in (("q_codes", p.B * p.Hq * p.N * p.d),
                              ("k_codes", p.B * p.Hkv * p.N * p.d), ("dq", p.B * p.Hq * Tm * 4),
                              ("dk", p.B * p.Hkv * Tn * 4), ("kbar", p.B * p.Hkv * p.d * 4),
-                             ("kbar_part", p.B * p.Hkv * 32 * p.d * 8),
                              ("k_sum64", p.B * p.Hkv * Tn * p.d * 8)):
             out[name] = off
             off += al(nbytes)

@@ -163,7 +163,10 @@ def test_predict_pool_then_select_equals_predict_mask(name):
         assert torch.equal(idx.view(-1, idx.shape[-1])[r, :n], i2.view(-1, i2.shape[-1])[r, :n])
     if w.qk_int8:
         reg = ws_regions(p)
-        a, b = reg["q_codes"], reg["kbar_part"]
+        a, b = reg["q_codes"], reg["kbar"] + 4 * p.B * p.Hkv * p.d
+        assert torch.equal(ws[a:b], ws2[a:b])
+        Tn = -(-p.N // p.bk)
+        a, b = reg["k_sum64"], reg["k_sum64"] + 8 * p.B * p.Hkv * Tn * p.d
         assert torch.equal(ws[a:b], ws2[a:b])
 
 
@@ -384,6 +387,30 @@ def test_int8_codes_on_half_integer_quotients():
     ws, *_ = gpu_predict(p, qd, qd)
     Q = q16.astype(np.float64)
     check_int8_state(ws, p, Q, Q)
+
+
+def test_int8_state_with_bf16_subnormal_keys():
+    """K values that are bf16 subnormals (below 2^-126), zero blocks and
+    normal values side by side: kbar is the float64 mean of every token,
+    rounded once, with no value flushed to zero; every code and scale
+    matches the oracle bit for bit (a subnormal delta takes the exact
+    division)."""
+    g = torch.Generator().manual_seed(11)
+    B, H, N, d = 1, 2, 1024 + 64, 128
+    q = torch.randn(B, H, N, d, generator=g)
+    k = torch.randn(B, H, N, d, generator=g)
+    k[:, 0] *= 2.0 ** -124                        # about a quarter below 2^-126
+    k[:, 1, ::7] *= 2.0 ** -130                   # subnormal tokens among normal ones
+    k[:, 1, 64:128] = 0.0                         # a whole key block of zeros
+    q[:, 1, 128:256] = 0.0                        # a whole query block of zeros
+    q16, k16 = q.to(torch.bfloat16), k.to(torch.bfloat16)
+    ksub = k16[:, 0].float().abs()
+    assert ((ksub > 0) & (ksub < 2.0 ** -126)).float().mean() > 0.1
+    w, _ = workload("llm_128k", N=N, Hq=H, Hkv=H)
+    p = params_for(w)
+    ws, *_ = gpu_predict(p, q16.to(dev()), k16.to(dev()))
+    Q, K = q16.double().numpy(), k16.double().numpy()
+    check_int8_state(ws, p, Q, K)
 
 
 def test_int8_with_fp16_io_and_ragged_tail():
