@@ -33,10 +33,29 @@ constexpr int kPoolMinBlocks = 4;  // <= 128 registers; a slab's rows take 64 of
 constexpr int kPoolBQ = 128;       // query block rows (the only b_q the library accepts)
 constexpr int kPoolBK = 64;        // key block rows
 
+// n / d for 0 <= n < 2^31 and a divisor 1 <= d < 2^31 known when the kernel
+// is launched, by a multiply (Granlund and Montgomery, "Division by invariant
+// integers using multiplication", 1994): with l = ceil(log2 d) and
+// m = floor(2^32 (2^l - d) / d) + 1, n / d = (umulhi(n, m) + n) >> l; the sum
+// stays below 2^32 because n < 2^31.
+struct FastDiv {
+  uint32_t mul, shr;
+  static FastDiv make(uint32_t d) {
+    uint32_t l = 0;
+    while ((uint64_t(1) << l) < d) ++l;
+    const uint64_t m = ((uint64_t(1) << 32) * ((uint64_t(1) << l) - d)) / d + 1;
+    return FastDiv{uint32_t(m), l};
+  }
+};
+__device__ __forceinline__ int fast_div(int n, uint32_t mul, uint32_t shr) {
+  return int((__umulhi(uint32_t(n), mul) + uint32_t(n)) >> shr);
+}
+
 struct PoolArgs {
   const void* q;
   const void* k;
   int32_t N, bq, bk, Tm, Tn;
+  uint32_t tm_mul, tm_shr, tn_mul, tn_shr;  // n / Tm and n / Tn by multiply (FastDiv)
   int64_t nQblocks;  // B*Hq*Tm: Q blocks come first in the pooling pass
   int64_t nblocks;   // blocks this pass visits
   float* q_mean;
@@ -61,8 +80,10 @@ __device__ __forceinline__ uint4 ld_stream(const void* p) {
 }
 
 // 16 bytes global -> shared, cached in L2 only; completed by cp_async_wait.
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
+// bytes is 16, or 0 to fill the 16 shared bytes with zeros and read nothing.
+__device__ __forceinline__ void cp_async16_zfill(void* smem, const void* gmem, uint32_t bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem)), "l"(gmem),
+               "r"(bytes)
                : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() {
@@ -228,13 +249,16 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
   constexpr int GQ = kPoolBQ / SLAB, GK = kPoolBK / SLAB;
   static_assert(WARPS % GQ == 0 && GQ % GK == 0, "groups must tile the CTA");
   static_assert(NR % CH == 0, "butterfly needs NR a multiple of CH");
-  __shared__ float part[WARPS][2 * D];
+  __shared__ __align__(16) float part[WARPS][2 * D];
   __shared__ float pmax[WARPS];
-  __shared__ double part64[SUM64 ? WARPS : 1][SUM64 ? D : 1];
+  __shared__ __align__(16) double part64[SUM64 ? WARPS : 1][SUM64 ? D : 1];
   __shared__ __align__(16) uint4 stage[PERSIST ? WARPS : 1][PERSIST ? NR : 1][32];
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = lane % CH, ro = lane / CH;
+  // this lane's eight columns of a warp's partial sums, as 16-byte words
+  auto part8 = [&](int w, int off) { return reinterpret_cast<float4*>(&part[w][off + c * 8]); };
+  auto part64_8 = [&](int w) { return reinterpret_cast<double2*>(&part64[w][c * 8]); };
   const int64_t nQw = a.nQblocks * GQ;
   const int64_t n_units = (nQw + (a.nblocks - a.nQblocks) * GK + WARPS - 1) / WARPS;
   // the slab that this warp takes in unit u: Q blocks first, then K blocks
@@ -262,7 +286,7 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
     if (KIND == 1) bid = nb - 1 - bid;
     const int T_ = sl.isQ ? a.Tm : a.Tn;
     const int BLK_ = sl.isQ ? kPoolBQ : kPoolBK;
-    const int bhi = bid / T_;
+    const int bhi = sl.isQ ? fast_div(bid, a.tm_mul, a.tm_shr) : fast_div(bid, a.tn_mul, a.tn_shr);
     sl.bh = bhi;
     sl.blk = bid - bhi * T_;
     sl.rows = min(BLK_, a.N - sl.blk * BLK_);
@@ -270,13 +294,20 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
     sl.row0 = sl.bh * a.N + int64_t(sl.blk) * BLK_ + sl.sub * SLAB;
     return sl;
   };
+  // rows past the slab's end are filled with zeros (their source address is
+  // the slab's block's first row, which every valid slab has, and is not read)
   auto prefetch = [&](const Slab& sl) {
     if (!PERSIST) return;
-    const uint16_t* src = static_cast<const uint16_t*>(sl.isQ ? a.q : a.k) + sl.row0 * D + c * 8;
+    if (sl.valid) {
+      const uint16_t* base = static_cast<const uint16_t*>(sl.isQ ? a.q : a.k);
+      const uint16_t* src = base + sl.row0 * D + c * 8;
+      const uint16_t* blk0 = base + (sl.row0 - sl.sub * SLAB) * D + c * 8;
 #pragma unroll
-    for (int u = 0; u < NR; ++u) {
-      const int r = ro + u * RPW;
-      if (r < sl.srows) cp_async16(&stage[warp][u][lane], src + int64_t(r) * D);
+      for (int u = 0; u < NR; ++u) {
+        const int r = ro + u * RPW;
+        const bool in = r < sl.srows;
+        cp_async16_zfill(&stage[warp][u][lane], in ? src + int64_t(r) * D : blk0, in ? 16u : 0u);
+      }
     }
     cp_async_commit();
   };
@@ -304,10 +335,7 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
   uint4 raw[NR];
   if constexpr (PERSIST) {
 #pragma unroll
-    for (int u = 0; u < NR; ++u) {
-      const int r = ro + u * RPW;
-      raw[u] = r < srows ? stage[warp][u][lane] : make_uint4(0, 0, 0, 0);
-    }
+    for (int u = 0; u < NR; ++u) raw[u] = stage[warp][u][lane];
   } else {
     const uint16_t* src = static_cast<const uint16_t*>(isQ ? a.q : a.k) + row0 * D + c * 8;
 #pragma unroll
@@ -424,28 +452,37 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
   // ---- the block's absmax and column sums over its G slabs (slab order)
   if (G > 1) {
     if (POOL && ro == 0) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) part[warp][c * 8 + e] = sx[e];
+      part8(warp, 0)[0] = make_float4(sx[0], sx[1], sx[2], sx[3]);
+      part8(warp, 0)[1] = make_float4(sx[4], sx[5], sx[6], sx[7]);
     }
     if (SUM64 && ro == 0) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) part64[warp][c * 8 + e] = s64[e];
+      for (int e = 0; e < 4; ++e) part64_8(warp)[e] = make_double2(s64[2 * e], s64[2 * e + 1]);
     }
     if (lane == 0) pmax[warp] = amax;
     named_barrier(1 + warp / G, 32 * G);
     if (POOL) {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) sx[e] = part[w0][c * 8 + e];
-      for (int g = 1; g < G; ++g)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) sx[e] += part[w0 + g][c * 8 + e];
+      float4 lo = part8(w0, 0)[0], hi = part8(w0, 0)[1];
+      for (int g = 1; g < G; ++g) {
+        const float4 l2 = part8(w0 + g, 0)[0], h2 = part8(w0 + g, 0)[1];
+        lo = make_float4(lo.x + l2.x, lo.y + l2.y, lo.z + l2.z, lo.w + l2.w);
+        hi = make_float4(hi.x + h2.x, hi.y + h2.y, hi.z + h2.z, hi.w + h2.w);
+      }
+      sx[0] = lo.x, sx[1] = lo.y, sx[2] = lo.z, sx[3] = lo.w;
+      sx[4] = hi.x, sx[5] = hi.y, sx[6] = hi.z, sx[7] = hi.w;
     }
     if (SUM64 && sub == 0) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) s64[e] = part64[w0][c * 8 + e];
-      for (int g = 1; g < G; ++g)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) s64[e] += part64[w0 + g][c * 8 + e];
+      for (int e = 0; e < 4; ++e) {
+        double2 t = part64_8(w0)[e];
+        for (int g = 1; g < G; ++g) {
+          const double2 t2 = part64_8(w0 + g)[e];
+          t.x += t2.x;
+          t.y += t2.y;
+        }
+        s64[2 * e] = t.x;
+        s64[2 * e + 1] = t.y;
+      }
     }
     amax = pmax[w0];
     for (int g = 1; g < G; ++g) amax = fmaxf(amax, pmax[w0 + g]);
@@ -497,15 +534,18 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
       for (int e = 0; e < 8; ++e) su[e] += __shfl_xor_sync(0xffffffffu, su[e], o);
     if (G > 1) {
       if (ro == 0) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) part[warp][D + c * 8 + e] = su[e];
+        part8(warp, D)[0] = make_float4(su[0], su[1], su[2], su[3]);
+        part8(warp, D)[1] = make_float4(su[4], su[5], su[6], su[7]);
       }
       named_barrier(1 + warp / G, 32 * G);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) su[e] = part[w0][D + c * 8 + e];
-      for (int g = 1; g < G; ++g)
-#pragma unroll
-        for (int e = 0; e < 8; ++e) su[e] += part[w0 + g][D + c * 8 + e];
+      float4 lo = part8(w0, D)[0], hi = part8(w0, D)[1];
+      for (int g = 1; g < G; ++g) {
+        const float4 l2 = part8(w0 + g, D)[0], h2 = part8(w0 + g, D)[1];
+        lo = make_float4(lo.x + l2.x, lo.y + l2.y, lo.z + l2.z, lo.w + l2.w);
+        hi = make_float4(hi.x + h2.x, hi.y + h2.y, hi.z + h2.z, hi.w + h2.w);
+      }
+      su[0] = lo.x, su[1] = lo.y, su[2] = lo.z, su[3] = lo.w;
+      su[4] = hi.x, su[5] = hi.y, su[6] = hi.z, su[7] = hi.w;
     }
     if (sub == 0) {
       float uu = 0.f;
@@ -515,10 +555,11 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
       for (int o = CH / 2; o > 0; o >>= 1) uu += __shfl_xor_sync(0xffffffffu, uu, o);
       float* mean = isQ ? a.q_mean : a.k_mean;
       if (lane < CH) {
-        const float n = float(rows);
+        // 1 / n is exact for a full block (a power of two), so this is sx / n
+        const float rn = 1.0f / float(rows);
         float4* dst = reinterpret_cast<float4*>(mean + (bh * T + blk) * D + c * 8);
-        dst[0] = make_float4(sx[0] / n, sx[1] / n, sx[2] / n, sx[3] / n);
-        dst[1] = make_float4(sx[4] / n, sx[5] / n, sx[6] / n, sx[7] / n);
+        dst[0] = make_float4(sx[0] * rn, sx[1] * rn, sx[2] * rn, sx[3] * rn);
+        dst[1] = make_float4(sx[4] * rn, sx[5] * rn, sx[6] * rn, sx[7] * rn);
       }
       if (lane == 0) (isQ ? a.s_q : a.s_k)[bh * T + blk] = uu / (float(rows) * float(rows));
     }
@@ -849,6 +890,11 @@ cudaError_t pool_impl(const sparge_params_t& p, const PredictPtrs& x, cudaStream
   pa.bk = p.bk;
   pa.Tm = int32_t(Tm);
   pa.Tn = int32_t(Tn);
+  const FastDiv dm = FastDiv::make(uint32_t(Tm)), dn = FastDiv::make(uint32_t(Tn));
+  pa.tm_mul = dm.mul;
+  pa.tm_shr = dm.shr;
+  pa.tn_mul = dn.mul;
+  pa.tn_shr = dn.shr;
   const int64_t nK = int64_t(p.B) * p.Hkv * Tn;
   pa.nQblocks = int64_t(p.B) * p.Hq * Tm;
   pa.nblocks = pa.nQblocks + nK;
