@@ -28,10 +28,17 @@
 namespace sparge {
 namespace {
 
-constexpr int kPoolThreads = 128;
-constexpr int kPoolMinBlocks = 4;  // <= 128 registers; a slab's rows take 64 of them
 constexpr int kPoolBQ = 128;       // query block rows (the only b_q the library accepts)
 constexpr int kPoolBK = 64;        // key block rows
+constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
+// Warps of a pooling CTA: at least four, and all the slabs of one query block.
+constexpr int pool_warps(int slab) { return kPoolBQ / slab > 4 ? kPoolBQ / slab : 4; }
+// CTAs per SM the register budget is set for: four 4-warp CTAs (128 registers;
+// a 32-row slab's rows take 64 of them), or two 8-warp CTAs.  (16-row slabs,
+// eight warps to a query block, ran the 128K pooling stage 35% slower than
+// 32-row slabs: the per-slab reductions and barriers cost more than the extra
+// warps hide.)
+constexpr int pool_min_blocks(int slab) { return pool_warps(slab) == 4 ? 4 : 2; }
 
 // n / d for 0 <= n < 2^31 and a divisor 1 <= d < 2^31 known when the kernel
 // is launched, by a multiply (Granlund and Montgomery, "Division by invariant
@@ -122,6 +129,26 @@ __device__ __forceinline__ uint32_t absmax2(uint32_t acc, uint32_t w) {
     asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(acc), "r"(w));
   else
     asm("max.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(r) : "r"(acc), "r"(w));
+  return r;
+}
+
+// Per-half max and min of packed 16-bit values (exact).
+template <bool BF16>
+__device__ __forceinline__ uint32_t max2_16(uint32_t a, uint32_t b) {
+  uint32_t r;
+  if (BF16)
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  else
+    asm("max.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+template <bool BF16>
+__device__ __forceinline__ uint32_t min2_16(uint32_t a, uint32_t b) {
+  uint32_t r;
+  if (BF16)
+    asm("min.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  else
+    asm("min.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
 
@@ -233,7 +260,8 @@ __device__ __forceinline__ double f64_scaled(float x) {
 //           sums in float64 (exact for 16-bit inputs), from which kbar is the
 //           float64 mean rounded once to float32.
 template <int D, bool BF16, int KIND, int SLAB>
-__global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(PoolArgs a) {
+__global__ void __launch_bounds__(32 * pool_warps(SLAB), pool_min_blocks(SLAB))
+    pool_kernel(PoolArgs a) {
   constexpr bool POOL = KIND != 1;
   constexpr bool SUM64 = KIND == 2;
   // The Q pass and the K code pass are persistent and stage the next unit in
@@ -244,11 +272,14 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
   constexpr int CH = D * 2 / 16;  // lanes per row
   constexpr int RPW = 32 / CH;    // rows per warp-wide load
   constexpr int NR = SLAB / RPW;  // rows per lane
-  constexpr int R = NR / CH;      // rows whose norm a lane holds after the butterfly
-  constexpr int WARPS = kPoolThreads / 32;
+  // after the butterfly a lane holds the norms of R rows, and each row's norm
+  // is held by SPREAD adjacent lanes
+  constexpr int R = NR >= CH ? NR / CH : 1;
+  constexpr int SPREAD = NR >= CH ? 1 : CH / NR;
+  constexpr int WARPS = pool_warps(SLAB);
   constexpr int GQ = kPoolBQ / SLAB, GK = kPoolBK / SLAB;
   static_assert(WARPS % GQ == 0 && GQ % GK == 0, "groups must tile the CTA");
-  static_assert(NR % CH == 0, "butterfly needs NR a multiple of CH");
+  static_assert(NR % CH == 0 || CH % NR == 0, "butterfly needs NR and CH nested");
   __shared__ __align__(16) float part[WARPS][2 * D];
   __shared__ float pmax[WARPS];
   __shared__ __align__(16) double part64[SUM64 ? WARPS : 1][SUM64 ? D : 1];
@@ -277,7 +308,7 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
     const int gw = gw64 < INT32_MAX ? int(gw64) : INT32_MAX;
     const int nqw = int(nQw);
     sl.isQ = KIND == 0 && gw < nqw;
-    const int lg = sl.isQ ? (GQ == 4 ? 2 : GQ == 2 ? 1 : 0) : (GK == 2 ? 1 : 0);
+    const int lg = sl.isQ ? ilog2(GQ) : ilog2(GK);
     const int rel = sl.isQ ? gw : gw - nqw;
     const int nb = int(sl.isQ ? a.nQblocks : a.nblocks - a.nQblocks);
     int bid = rel >> lg;
@@ -389,18 +420,24 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
     amax = absmax2_value<BF16>(absmax2<BF16>(absmax2<BF16>(am2[0], am2[1]),
                                              absmax2<BF16>(am2[2], am2[3])));
     // ---- butterfly over the CH lanes of a row: at offset o the lanes with
-    // bit o set keep the upper half of their rows and send the lower half
+    // bit o set keep the upper half of their rows and send the lower half;
+    // once a lane is down to one row, the remaining offsets add plainly
 #pragma unroll
-    for (int o = CH / 2, cnt = NR; o > 0; o >>= 1, cnt >>= 1) {
+    for (int o = CH / 2; o > 0; o >>= 1) {
       const bool up = (lane & o) != 0;
+      const int cnt = NR * 2 * o / CH;  // rows carried into this step (< 2: one)
+      if (cnt >= 2) {
 #pragma unroll
-      for (int k = 0; k < cnt / 2; ++k) {
-        const float send = up ? v[k] : v[k + cnt / 2];
-        const float keep = up ? v[k + cnt / 2] : v[k];
-        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        for (int k = 0; k < cnt / 2; ++k) {
+          const float send = up ? v[k] : v[k + cnt / 2];
+          const float keep = up ? v[k + cnt / 2] : v[k];
+          v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+      } else {
+        v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
       }
     }
-    // lane c of a row group now holds rows c * R .. c * R + R - 1
+    // lane c of a row group now holds rows (c / SPREAD) * R .. + R - 1
 #pragma unroll
     for (int t = 0; t < R; ++t) inv_own[t] = v[t] > 0.f ? rsqrtf(v[t]) : 0.f;
     if (SUM64) {
@@ -420,16 +457,29 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
       }
     }
   } else {
+    // max |fl(x - kbar)| over the rows from each column's max and min of x:
+    // rounding is monotone, so fl(xmin - kbar) <= fl(x - kbar) <= fl(xmax -
+    // kbar) for every row, and the larger magnitude of those two is the max
+    // (a lane's rows are valid in order: row u is valid only if row 0 is)
+    uint32_t hi2[4], lo2[4];
 #pragma unroll
     for (int u = 0; u < NR; ++u) {
       if (ro + u * RPW < srows) {
         const uint32_t w[4] = {raw[u].x, raw[u].y, raw[u].z, raw[u].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          float d0, d1;
-          unpack2(add2(widen2<BF16>(w[e]), nkb2[e]), d0, d1);
-          amax = fmaxf(amax, fmaxf(fabsf(d0), fabsf(d1)));
+          hi2[e] = u == 0 ? w[e] : max2_16<BF16>(hi2[e], w[e]);
+          lo2[e] = u == 0 ? w[e] : min2_16<BF16>(lo2[e], w[e]);
         }
+      }
+    }
+    if (ro < srows) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float a0, a1, b0, b1;
+        unpack2(add2(widen2<BF16>(hi2[e]), nkb2[e]), a0, a1);
+        unpack2(add2(widen2<BF16>(lo2[e]), nkb2[e]), b0, b1);
+        amax = fmaxf(amax, fmaxf(fmaxf(fabsf(a0), fabsf(a1)), fmaxf(fabsf(b0), fabsf(b1))));
       }
     }
   }
@@ -514,7 +564,7 @@ __global__ void __launch_bounds__(kPoolThreads, kPoolMinBlocks) pool_kernel(Pool
 #pragma unroll
     for (int e = 0; e < 4; ++e) x2[e] = widen2<BF16>(w[e]);
     if (POOL) {
-      const float iv = __shfl_sync(0xffffffffu, inv_own[u % R], group_base | (u / R));
+      const float iv = __shfl_sync(0xffffffffu, inv_own[u % R], group_base | ((u / R) * SPREAD));
       const uint64_t iv2 = pack2(iv, iv);
 #pragma unroll
       for (int e = 0; e < 4; ++e) su2[e] = fma2(x2[e], iv2, su2[e]);
@@ -871,10 +921,12 @@ cudaError_t launch_pool(const PoolArgs& pa, int64_t warps, cudaStream_t s) {
                            cudaFuncAttributePreferredSharedMemoryCarveout,
                            int(cudaSharedmemCarveoutMaxShared));
   if (e != cudaSuccess) return e;
-  const int64_t units = cdiv(warps, kPoolThreads / 32);
-  const int64_t ctas =
-      KIND == 2 ? units : std::max<int64_t>(1, std::min<int64_t>(units, int64_t(sms) * kPoolMinBlocks));
-  pool_kernel<D, BF16, KIND, SLAB><<<unsigned(ctas), kPoolThreads, 0, s>>>(pa);
+  constexpr int WARPS = pool_warps(SLAB);
+  const int64_t units = cdiv(warps, WARPS);
+  const int64_t ctas = KIND == 2 ? units
+                                 : std::max<int64_t>(1, std::min<int64_t>(
+                                                            units, int64_t(sms) * pool_min_blocks(SLAB)));
+  pool_kernel<D, BF16, KIND, SLAB><<<unsigned(ctas), 32 * WARPS, 0, s>>>(pa);
   return cudaGetLastError();
 }
 
@@ -907,10 +959,12 @@ cudaError_t pool_impl(const sparge_params_t& p, const PredictPtrs& x, cudaStream
   pa.status = x.status;
   cudaError_t e;
   constexpr int SLAB = D == 128 ? 32 : 64;  // 8 KB of bf16/f16 per warp
-  constexpr int64_t GQ = kPoolBQ / SLAB, GK = kPoolBK / SLAB;
+  constexpr int SLAB_Q = SLAB;  // the pooling pass's slab (any power of two from 16 works)
+  constexpr int64_t GK = kPoolBK / SLAB;
+  constexpr int64_t GQq = kPoolBQ / SLAB_Q, GKq = kPoolBK / SLAB_Q;
   if (x.k_codes == nullptr) {
     // one pass over Q then K blocks
-    return launch_pool<D, BF16, 0, SLAB>(pa, pa.nQblocks * GQ + nK * GK, s);
+    return launch_pool<D, BF16, 0, SLAB_Q>(pa, pa.nQblocks * GQq + nK * GKq, s);
   }
   if constexpr (D != 128) {
     return cudaErrorInvalidValue;  // the INT8 path exists for d = 128 only
@@ -933,7 +987,7 @@ cudaError_t pool_impl(const sparge_params_t& p, const PredictPtrs& x, cudaStream
   if ((e = launch_pool<D, BF16, 1, SLAB>(ca, nK * GK, s)) != cudaSuccess) return e;
   PoolArgs qa = pa;
   qa.nblocks = qa.nQblocks;
-  return launch_pool<D, BF16, 0, SLAB>(qa, qa.nQblocks * GQ, s);
+  return launch_pool<D, BF16, 0, SLAB_Q>(qa, qa.nQblocks * GQq, s);
   }
 }
 
