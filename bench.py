@@ -231,7 +231,7 @@ def run_native(args, rank, world, local_rank):
     p = fb.make_params(w.B, w.Hq, w.Hkv, w.N, w.d, w.tau, w.theta, w.lam, causal=w.causal,
                        qk_int8=w.qk_int8, io_dtype=tdt)
     ws = fb.workspace(p, dev)
-    mask, idx, cnt, _, _ = fb.predict_outputs(p, dev)
+    mask, idx, cnt, sq_out, _ = fb.predict_outputs(p, dev)
     o = torch.empty(q.shape, dtype=tdt, device=dev)
     stats = torch.zeros(5, dtype=torch.int64, device=dev)
     perm = hws = None
@@ -292,6 +292,10 @@ def run_native(args, rank, world, local_rank):
     st = stats.cpu().numpy().astype(np.int64)
     if fb.sparge_device_status(ws) != 0:
         raise RuntimeError("device status reported an error")
+    # the select stage's own work on this step's pooled statistics (untimed)
+    fb.sparge_predict_select(p, mask, idx, cnt, sq_out, None, ws, stream)
+    torch.cuda.synchronize()
+    sel_work = select_work(w, sq_out.cpu().numpy(), int(cnt.sum()), w.theta)
     mask_h0 = mask[:, 0].cpu().numpy().astype(bool) if rank == 0 else None
 
     sampler = ClockSampler(_gpu_uuid(torch, dev)) if local_rank == 0 or world > 1 else None
@@ -353,6 +357,10 @@ def run_native(args, rank, world, local_rank):
         step(q, k, v, o, prm=ps)
         torch.cuda.synchronize()
         sst = [int(x) for x in stats.cpu()]
+        fb.sparge_predict_select(ps, mask, idx, cnt, sq_out, None, ws, stream)
+        torch.cuda.synchronize()
+        s_sel_work = select_work(w, sq_out.cpu().numpy(), int(cnt.sum()), -1.0)
+        pk, _ = load_peaks()
         sper = [(ev(), ev(), ev(), ev()) for _ in range(args.steps)]
         sspan = [(ev(), ev()) for _ in range(args.steps)]
         for s_ in range(args.steps):
@@ -368,12 +376,15 @@ def run_native(args, rank, world, local_rank):
         s_step = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in sspan])), world, dev)
         s_attn = float(np.mean([a.elapsed_time(b) for (_, _, a, b) in sper]))
         s_pred = float(np.mean([a.elapsed_time(c) for (a, _, c, _) in sper]))
+        s_sel = float(np.mean([b.elapsed_time(c) for (_, b, c, _) in sper]))
         vis = _visible_blocks(w)
         sparse = {
             "tau": 0.5, "theta": -1.0, "lambda": w.lam, "steps": args.steps,
             "value": round(aggregate_tops(world, dense_equiv_ops(w), 1, s_step), 3), "unit": "TOPS",
             "latency_ms": {"step": round(s_step, 4), "predict": round(s_pred, 4),
-                           "attention": round(s_attn, 4)},
+                           "predict_select": round(s_sel, 4), "attention": round(s_attn, 4)},
+            "select_roofline": select_roofline(s_sel_work, s_sel, fp32_peak_tflops(pk),
+                                               float(pk["hbm_gbs"])),
             "sparsity": {"mg": round(1.0 - sst[1] / vis, 6),
                          "pv_slices_skipped": round(sst[4] / max(1, sst[3] + sst[4]), 6),
                          "total": round(1.0 - (sst[1] + sst[3] / 4.0) / (2.0 * vis), 6)},
@@ -486,7 +497,6 @@ def run_native(args, rank, world, local_rank):
     traffic = profiled_traffic(w.name, w.N)
     pbytes = pool_bytes(w)
     hbm_peak = float(peaks["hbm_gbs"])
-    sel_flops = 2.0 * w.d * _visible_pairs(w)
     fp32_peak = fp32_peak_tflops(peaks)
     sparsity = {
         "mg": round(1.0 - qk_blocks / vis, 6),
@@ -530,12 +540,7 @@ def run_native(args, rank, world, local_rank):
                                     "kernel": "scatter of O back to token order: read once, "
                                               "written once / stage time"}}
                if w.grid else {}),
-            "select": {"bound": "fp32", "achieved": round(sel_flops / (sel_ms * 1e-3) / 1e12, 2),
-                       "peak": round(fp32_peak, 1), "unit": "TFLOP/s",
-                       "frac": round(sel_flops / (sel_ms * 1e-3) / 1e12 / fp32_peak, 4),
-                       "flops_per_launch": sel_flops,
-                       "kernel": "select_kernel: 2*d flops per visible (i, j) for S_hat; "
-                                 "peak = 148 SMs x 128 FP32 lanes x 2 x max SM clock"},
+            "select": select_roofline(sel_work, sel_ms, fp32_peak, hbm_peak),
         },
         "sparsity": sparsity,
         "work": {"tiles": tiles, "qk_blocks": qk_blocks, "pv_blocks": pv_blocks,
@@ -584,9 +589,52 @@ def _gpu_uuid(torch, dev):
         return str(dev.index)
 
 
-def _visible_pairs(w):
-    """(query block, key block) pairs the select stage scores: causal-visible."""
-    return _visible_blocks(w)
+def _visible_per_row(w):
+    """Visible key blocks of each query block (all of them unless causal)."""
+    Tm, Tn = -(-w.N // w.bq), -(-w.N // w.bk)
+    if not w.causal:
+        return np.full(Tm, Tn, dtype=np.int64)
+    last = np.minimum(w.N, (np.arange(Tm) + 1) * w.bq) - 1
+    return np.minimum(Tn, last // w.bk + 1).astype(np.int64)
+
+
+def select_work(w, s_q, kept, theta):
+    """The select stage's algorithmic work on one step: S_hat's 2*d flops for
+    every visible (i, j) of a query block that is not a fix block (Eq. 9: a
+    fix block's row is all ones and its S_hat decides nothing), and its HBM
+    bytes: the block means and self-similarities read once, the mask, the
+    kept entries of the skip list and the counts written."""
+    Tm, Tn = -(-w.N // w.bq), -(-w.N // w.bk)
+    vis = _visible_per_row(w)
+    nonfix = np.asarray(s_q).reshape(w.B * w.Hq, Tm) >= theta
+    pairs = int((nonfix * vis[None, :]).sum())
+    nbytes = (4 * (w.B * w.Hq * Tm * (w.d + 1) + w.B * w.Hkv * Tn * (w.d + 1))
+              + w.B * w.Hq * Tm * Tn + 4 * kept + 4 * w.B * w.Hq * Tm)
+    return {"flops": 2.0 * w.d * pairs, "bytes": float(nbytes),
+            "nonfix_rows": int(nonfix.sum()), "rows": int(nonfix.size)}
+
+
+def select_roofline(work, ms, fp32_peak, hbm_peak):
+    """Roofline of the select stage: its S_hat flops against the FP32 FMA
+    peak and its bytes against HBM; the larger of the two ideal times bounds
+    the stage."""
+    t_f = work["flops"] / (fp32_peak * 1e12)
+    t_b = work["bytes"] / (hbm_peak * 1e9)
+    sec = ms * 1e-3
+    if t_f >= t_b:
+        out = {"bound": "fp32", "achieved": round(work["flops"] / sec / 1e12, 2),
+               "peak": round(fp32_peak, 1), "unit": "TFLOP/s"}
+    else:
+        out = {"bound": "hbm", "achieved": round(work["bytes"] / sec / 1e9, 1),
+               "peak": hbm_peak, "unit": "GB/s"}
+    out.update({"frac": round(max(t_f, t_b) / sec, 4), "flops_per_launch": work["flops"],
+                "bytes_per_launch": work["bytes"], "nonfix_rows": work["nonfix_rows"],
+                "rows": work["rows"],
+                "kernel": "select_kernel: 2*d flops per visible (i, j) of a non-fix query "
+                          "block for S_hat (peak 148 SMs x 128 FP32 lanes x 2 x max SM "
+                          "clock), bytes: means and self-similarities read, mask, kept "
+                          "skip-list entries and counts written"})
+    return out
 
 
 def _visible_blocks(w):

@@ -11,6 +11,7 @@ import os
 import subprocess
 import sys
 
+import numpy as np
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -60,6 +61,23 @@ def test_visible_blocks_causal_count():
     # causal: query block i (128 rows) sees key blocks 0 .. 2i+1 (64 rows each)
     w = get_workload("llm_32k").replace(N=1024, Hq=1, Hkv=1)
     assert bench._visible_blocks(w) == sum(2 * i + 2 for i in range(8))
+
+
+def test_select_work_counts_only_non_fix_rows():
+    # causal, b_q 128, b_k 64, N 512: query blocks see 2, 4, 6, 8 key blocks.
+    # Head 0's last query block and head 1's first (s exactly theta: Eq. 9's
+    # strict <) are not fix blocks, so S_hat is needed for 8 + 2 visible pairs.
+    w = get_workload("llm_32k", N=512, Hq=2, Hkv=1)
+    s_q = np.array([[[0.1, 0.1, 0.1, 0.9]], [[0.5, 0.2, 0.4999, 0.1]]]).reshape(1, 2, 4)
+    work = bench.select_work(w, s_q, kept=17, theta=0.5)
+    assert work["flops"] == 2 * 128 * (8 + 2)
+    assert work["nonfix_rows"] == 2 and work["rows"] == 8
+    means = 4 * (2 * 4 * 129 + 1 * 8 * 129)      # block means + self-similarities read
+    writes = 2 * 4 * 8 + 4 * 17 + 4 * 2 * 4      # mask, kept skip-list entries, counts
+    assert work["bytes"] == means + writes
+    # every block a fix block: no flops, bound by the bytes
+    r = bench.select_roofline(bench.select_work(w, s_q, 17, theta=2.0), 1e-3, 74.4, 6550.4)
+    assert r["bound"] == "hbm" and r["flops_per_launch"] == 0
 
 
 def test_fp32_peak_from_unit_counts():
