@@ -669,9 +669,9 @@ struct SelectArgs {
   float tau, theta, scale;
 };
 
-// e * 2^40 as an integer (e in [0, 1]); exact for e >= 2^-16
-__device__ __forceinline__ unsigned long long fixed40(float e) {
-  return __float2ull_rz(e * 1099511627776.0f);
+// e * 2^38 as an integer (e in [0, 1]); exact for e >= 2^-14
+__device__ __forceinline__ unsigned long long fixed38(float e) {
+  return __float2ull_rz(e * 274877906944.0f);
 }
 
 __device__ __forceinline__ int visible_cols(int i, int N, int bq, int bk, int Tn, int causal) {
@@ -801,15 +801,15 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   // unnormalised softmax weights; -1 marks a -inf entry.  Each weight's mass
-  // is also taken as the integer e * 2^40 (exact for e >= 2^-16, below that
-  // truncated by < 2^-40), so that every partial sum below is exact and does
+  // is also taken as the integer e * 2^38 (exact for e >= 2^-14, below that
+  // truncated by < 2^-38), so that every partial sum below is exact and does
   // not depend on the order of summation.
   unsigned long long tot = 0ull;
   for (int j = lane; j < nvis; j += 32) {
     const float v = row[j];
     const float e = (v == -INFINITY) ? -1.f : expf(v - mx);
     row[j] = e;
-    if (e >= 0.f) tot += fixed40(e);
+    if (e >= 0.f) tot += fixed38(e);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
@@ -823,27 +823,36 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(SelectArgs a) {
     // where the running sum from the top reaches the target.
     const unsigned long long target =
         static_cast<unsigned long long>(ceil(double(a.tau) * double(tot)));
-    unsigned long long* hist = reinterpret_cast<unsigned long long*>(ks) + w * 256;
+    // the warp's 256-bucket histogram of masses, as two 32-bit halves (the low
+    // 19 bits of each mass and the rest, at most 2^19: a bucket's sums stay
+    // below 5952 * 2^19 < 2^32 for the longest rows the library accepts), so
+    // that every update is a native 32-bit shared atomic, not a 64-bit one
+    uint32_t* hist_lo = reinterpret_cast<uint32_t*>(ks) + w * 512;
+    uint32_t* hist_hi = hist_lo + 256;
     uint32_t prefix = 0u;
     unsigned long long above = 0ull;  // mass of the entries above the prefix's range
 #pragma unroll 1
     for (int shift = 24; shift >= 0; shift -= 8) {
       const uint32_t pmask = shift == 24 ? 0u : (0xFFFFFFFFu << (shift + 8));
 #pragma unroll
-      for (int b = 0; b < 8; ++b) hist[lane * 8 + b] = 0ull;
+      for (int b = 0; b < 8; ++b) hist_lo[lane * 8 + b] = hist_hi[lane * 8 + b] = 0u;
       __syncwarp();
       for (int j = lane; j < nvis; j += 32) {
         const float e = row[j];
         const uint32_t key = __float_as_uint(e);
-        if (e >= 0.f && (key & pmask) == prefix)
-          atomicAdd(hist + ((key >> shift) & 255u), fixed40(e));
+        if (e >= 0.f && (key & pmask) == prefix) {
+          const unsigned long long m = fixed38(e);
+          const uint32_t bin = (key >> shift) & 255u;
+          atomicAdd(hist_lo + bin, uint32_t(m & 0x7FFFFull));
+          atomicAdd(hist_hi + bin, uint32_t(m >> 19));
+        }
       }
       __syncwarp();
       // lane L holds digits 8L .. 8L+7; suffix sums over lanes from the top
       unsigned long long h[8], mine = 0ull;
 #pragma unroll
       for (int b = 0; b < 8; ++b) {
-        h[b] = hist[lane * 8 + b];
+        h[b] = (static_cast<unsigned long long>(hist_hi[lane * 8 + b]) << 19) + hist_lo[lane * 8 + b];
         mine += h[b];
       }
       unsigned long long incl = mine;  // mass of lanes >= this lane
