@@ -132,7 +132,10 @@ sparge_status_t sparge_inverse_permute(const void* y, void* x, int32_t B, int32_
  *          first kv_cnt entries valid (the rest are left unspecified)
  *   kv_cnt [B, Hq, T_m] int32
  *   s_q    [B, Hq, T_m] float, s_k [B, Hkv, T_n] float (both nullable)
- * With qk_int8 it also quantises Q and K - mean(K) per block into ws. */
+ * With qk_int8 it also quantises Q and K - mean(K) per block into ws
+ * (Algorithm 1 step 2): mean(K) is the per-head mean over all N tokens, summed
+ * in float64 and rounded once to float32; per block delta = absmax / 127 and
+ * code = round-half-even(x / delta) of the IEEE float32 quotient. */
 sparge_status_t sparge_predict_mask(const sparge_params_t* p, const void* q, const void* k,
                                     uint8_t* mask, int32_t* kv_idx, int32_t* kv_cnt, float* s_q,
                                     float* s_k, void* ws, size_t ws_bytes, cudaStream_t stream);
