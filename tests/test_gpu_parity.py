@@ -11,7 +11,7 @@ import torch
 
 import free_block_sparse_predict_b200 as fb
 from oracle import sparge_oracle as orc
-from synth import bf16_bits_from_f32, to_f32
+from synth import bf16_bits_from_f32, to_f32, to_f64
 
 from gpu_common import (INT8_COS, INT8_REL_L1, MAX_ABS, MEAN_REL_L1, check_mask,
                         compare_rows, dev, gpu_attention, gpu_compact, gpu_predict,
@@ -539,6 +539,30 @@ def test_maximum_length_mask_and_sampled_tiles():
     assert mx <= MAX_ABS and l1 <= MEAN_REL_L1, (mx, l1, ost["near_lambda"])
     # one more key block is refused before anything runs
     assert fb.sparge_workspace_bytes(params_for(w.replace(N=N + 1))) == 0
+
+
+def test_maximum_length_selective_rows_and_constant_scores():
+    """The TopCdf radix select on the longest rows the library accepts (5952
+    key blocks): theta = -1 makes every query block selective and tau = 0.5
+    makes TopCdf cut.  Head 1 has Q = 0, so every score of its rows is equal
+    and every weight is 1: the histogram's largest bucket sums (5952 weights
+    of 2^38 in two 32-bit halves) and TopCdf's ties (all entries equal the cut
+    value, so all are kept, Eq. 8's reading)."""
+    N = 5952 * 64
+    w, t = workload("llm_32k", N=N, Hq=2, Hkv=1)
+    w = w.replace(theta=-1.0, tau=0.5)
+    q = t["q"].copy()
+    q[:, 1] = 0
+    Q, K = to_f64(q, w.dtype), to_f64(t["k"], w.dtype)
+    p = params_for(w)
+    ws, mask, idx, cnt, sq, sk = gpu_predict(p, to_dev(q, w.dtype), to_dev(t["k"], w.dtype))
+    pr = orc.predict_mask(Q, K, w.bq, w.bk, w.tau, w.theta, w.causal, w.scale)
+    M = mask.cpu().numpy().astype(bool)
+    check_mask(M, pr, "maximum length, theta -1, tau 0.5")
+    vis = pr["visible"]
+    assert np.array_equal(M[0, 1], vis)          # constant rows keep every visible block
+    assert M[0, 0].sum() < 0.9 * vis.sum()       # selective rows drop blocks
+    assert int(cnt.view(-1)[-1]) == M[0, 1, -1].sum() == 5952
 
 
 @pytest.mark.parametrize("N,causal", [(1, False), (1, True), (65, True), (129, False),
