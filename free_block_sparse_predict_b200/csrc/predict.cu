@@ -1,11 +1,13 @@
 // Stage 1 of SpargeAttn: the sparse-block predictor (paper review page,
 // section 三, Eq. 4-9 and Algorithm 1 steps 2-5).
 //
-//   pool_kernel<.., 0>  one pass over Q and K (HBM bound), one warp per
-//                   64-row slab held in registers: the mean token (Eq. 4, 5) and the self-similarity
-//                   CosSim (Eq. 6, read as the mean of the block's token cosine
-//                   matrix), via mean_{a,b} xh_a.xh_b = |sum_a xh_a|^2 / n^2.
-//                   With INT8 it also quantises Q per block (Algorithm 1 step 2).
+//   pool_kernel<.., 0>  one pass over Q (and, without INT8, K; HBM bound),
+//                   one warp per slab of 32 rows (64 at d = 64) held in
+//                   registers: the mean token (Eq. 4, 5) and the
+//                   self-similarity CosSim (Eq. 6, read as the mean of the
+//                   block's token cosine matrix), via
+//                   mean_{a,b} xh_a.xh_b = |sum_a xh_a|^2 / n^2.  With INT8 it
+//                   also quantises Q per block (Algorithm 1 step 2).
 //   pool_kernel<.., 2>  with INT8, the pooling pass over K alone, which also
 //                   writes each K block's float64 column sums;
 //   kbar_kernel     per-head mean of K from them (K smoothing);
@@ -239,8 +241,8 @@ __device__ __forceinline__ double f64_scaled(float x) {
 // is processed, so every byte of Q and K is read from HBM exactly once per
 // pass.  A CTA of four warps takes units of four slabs (one Q block or two K
 // blocks); the Q pass and the K code pass are persistent, taking units in a
-// grid-stride loop, and each warp
-// copies its slab of the next unit into its shared-memory buffer (cp.async)
+// grid-stride loop, and each warp copies its slab of the next unit into its
+// shared-memory buffer (cp.async; rows past a ragged end are zero-filled)
 // while it works on the current one, so loads stay in flight all the time.
 // Lane (ro, c) owns the 16-byte chunk c of rows ro, ro + RPW, ...  Arithmetic
 // runs on packed fp32 pairs in two sweeps over the registers: the first takes
